@@ -1,0 +1,10 @@
+"""CPU oracle for the skip-softmax / N:M sparse attention forward.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The product path
+(``softmax_ssa_fwd_b200``) never imports it and shares no code with it.
+
+The arithmetic lives in ``ssa_oracle.c`` (plain C, fp64); this module only
+compiles it (``build()``) and marshals numpy arrays into it (``run_items``).
+"""
+from .oracle import build, lib_path, run_items, visited_tiles, OracleResult  # noqa: F401
