@@ -1,0 +1,113 @@
+/*
+ * ssa.h -- C ABI of libssa: the skip-softmax / N:M sparse flash-attention
+ * forward pass on NVIDIA B200 (sm_100a).
+ *
+ * The method (cited by page title and section):
+ *   - "Skip-Softmax Sparse Attention for Diffusion Models" (Model-Optimizer
+ *     examples/diffusers/sparsity README), intro: skip-softmax (BLASST) skips
+ *     KV tiles whose attention scores are negligible during the FlashAttention
+ *     computation; "Threshold Modes" table: the kernel receives the lambda
+ *     threshold and compares in the log2 domain (log2(lambda)).  A (Br x Bc)
+ *     tile is skipped when exp(tile_row_max - running_max) < lambda holds for
+ *     every query row of the tile; a skipped tile issues no exp, no V load and
+ *     no P.V product, and leaves the running max, sum and output untouched.
+ *   - "Attention Sparsity for HuggingFace Models" (Model-Optimizer
+ *     examples/llm_sparsity/attention_sparsity README), "N:M Sparse Softmax"
+ *     and "Custom N:M configuration": for every M consecutive key positions
+ *     keep the top-N scores and set the rest to -inf before softmax
+ *     (M = 4 with N = 1..3, M = 8 with N = 1..7); the first
+ *     dense_sink_tokens keys and a local window of dense_recent_tokens keys
+ *     are kept dense; tile shape knobs br / bc.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *     16-byte aligned, contiguous, owned by the caller.  The library keeps no
+ *     reference to them after the call returns.
+ *   - q:   [B, Lq, Hq, d]  bf16
+ *     k,v: [B, Lk, Hkv, d] bf16
+ *     out: [B, Lq, Hq, d]  bf16 (overwritten)
+ *     lse: [B, Hq, Lq]     fp32, natural-log log-sum-exp of the scaled scores
+ *                          of the kept keys (-inf for a row with none)
+ *     tile_skip_count: [B, Hq, nQ] int32, nQ = ceil(Lq / Br): number of
+ *                          visited key tiles skipped by each query tile
+ *                          (overwritten, not accumulated).
+ *   - Query head hq reads KV head hq / (Hq / Hkv) (grouped-query attention).
+ *   - causal != 0: bottom-right aligned mask, query row i sees keys
+ *     j <= i + (Lk - Lq).  Key tiles wholly above the diagonal are never
+ *     visited and are not counted.
+ *   - scores are scale * q.k; scale > 0 and finite.
+ *   - mode: bit 0 (SSA_MODE_SKIP) enables the tile skip with threshold
+ *     lambda (>= 0; 0 never skips); bit 1 (SSA_MODE_NM) enables N:M with
+ *     n, m, sink, recent.  Parameters of a disabled mode are ignored.
+ *     N:M groups are aligned to key 0; the recent window of row i is the keys
+ *     0 <= pos_i - j < recent.  n == m is accepted (it keeps every key).
+ *   - Br, Bc in {64, 128}; d in {64, 128}.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  Argument errors are reported synchronously,
+ *     before anything is launched; no exception crosses this boundary.
+ *   - A device-side wait that times out (it never should) makes the kernel
+ *     unwind and record SSA_ERR_TIMEOUT in a per-device status word, read by
+ *     ssa_device_status().
+ */
+#ifndef SSA_H
+#define SSA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SSA_OK 0
+#define SSA_ERR_INVALID_ARG (-1) /* null pointer, non-positive size, bad lambda/scale, misalignment */
+#define SSA_ERR_UNSUPPORTED (-2) /* d, Br, Bc, n/m outside the supported set */
+#define SSA_ERR_CUDA (-3)        /* a CUDA runtime/driver call failed (launch, tensor map) */
+#define SSA_ERR_TIMEOUT (-4)     /* a device-side bounded wait expired */
+
+#define SSA_MODE_DENSE 0
+#define SSA_MODE_SKIP 1
+#define SSA_MODE_NM 2
+
+/* Forward pass.  Returns SSA_OK once the kernel is enqueued, or a negative
+ * status (nothing enqueued) for invalid or unsupported arguments. */
+int ssa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+            int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
+            float scale, int mode, float lambda, int n, int m, int sink, int recent, int Br, int Bc,
+            void* stream);
+
+/* Same kernel as ssa_fwd, also writing per-tile evidence (either may be NULL):
+ *   skip_bits: [B, Hq, nQ, ceil(nK / 32)] uint32, nK = ceil(Lk / Bc); bit kt of
+ *              query tile qt is set iff key tile kt was visited and skipped.
+ *              Every word of every query tile is written.
+ *   keep_bits: [B, Hq, Lq, ceil(Lk / 32)] uint32; bit j of row i is set iff key
+ *              j is visible to row i and kept by N:M (every visible key when N:M
+ *              is off), for the key tiles the row's query tile visits.  Words of
+ *              tiles that are not visited are not written: zero the buffer first.
+ * Skipped tiles still report their keep bits (the N:M mask precedes the skip). */
+int ssa_fwd_debug(const void* q, const void* k, const void* v, void* out, float* lse,
+                  int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                  int causal, float scale, int mode, float lambda, int n, int m, int sink,
+                  int recent, int Br, int Bc, void* stream, uint32_t* skip_bits,
+                  uint32_t* keep_bits);
+
+/* Total key tiles visited by all query tiles of one (batch, head) pair: a pure
+ * function of the shape, used to turn skip counts into skip fractions and
+ * executed FLOPs.  Returns -1 for invalid sizes. */
+int64_t ssa_visited_tiles(int causal, int Lq, int Lk, int Br, int Bc);
+
+/* Synchronises `stream`, returns SSA_OK or SSA_ERR_TIMEOUT if a kernel on this
+ * device recorded a timed-out wait since the last call, and clears the word.
+ * Returns SSA_ERR_CUDA if the synchronisation itself fails. */
+int ssa_device_status(void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* ssa_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int ssa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H */

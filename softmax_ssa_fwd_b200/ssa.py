@@ -1,0 +1,135 @@
+"""Thin ctypes binding of libssa (include/ssa.h): argument marshalling only.
+
+Every step of the attention runs in the CUDA kernels behind the C ABI.  The
+binding raises if the library cannot be loaded; there is no CPU fallback.
+Functions keep the C names; tensors are passed as torch CUDA tensors (their
+device pointers are handed to the library) and the stream defaults to torch's
+current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssa.so")
+
+SSA_OK = 0
+SSA_ERR_INVALID_ARG = -1
+SSA_ERR_UNSUPPORTED = -2
+SSA_ERR_CUDA = -3
+SSA_ERR_TIMEOUT = -4
+MODE_DENSE, MODE_SKIP, MODE_NM = 0, 1, 2
+
+EXPORTED = ["ssa_fwd", "ssa_fwd_debug", "ssa_visited_tiles", "ssa_device_status",
+            "ssa_status_string", "ssa_version"]
+
+
+class SSAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libssa.so not built at {LIB_PATH}; run softmax_ssa_fwd_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    fwd_args = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, F, I, I, I, I, I, I, P]
+    lib.ssa_fwd.restype = I
+    lib.ssa_fwd.argtypes = fwd_args
+    lib.ssa_fwd_debug.restype = I
+    lib.ssa_fwd_debug.argtypes = fwd_args + [P, P]
+    lib.ssa_visited_tiles.restype = ctypes.c_int64
+    lib.ssa_visited_tiles.argtypes = [I, I, I, I, I]
+    lib.ssa_device_status.restype = I
+    lib.ssa_device_status.argtypes = [P]
+    lib.ssa_status_string.restype = ctypes.c_char_p
+    lib.ssa_status_string.argtypes = [I]
+    lib.ssa_version.restype = I
+    lib.ssa_version.argtypes = []
+    return lib
+
+
+lib = _load()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return stream
+
+
+def status_string(status: int) -> str:
+    return lib.ssa_status_string(int(status)).decode()
+
+
+def ssa_version() -> int:
+    return lib.ssa_version()
+
+
+def ssa_visited_tiles(causal, Lq, Lk, Br, Bc) -> int:
+    return int(lib.ssa_visited_tiles(int(causal), Lq, Lk, Br, Bc))
+
+
+def ssa_device_status(stream=None) -> int:
+    return lib.ssa_device_status(_stream(stream))
+
+
+def ssa_fwd(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode, lam,
+            n, m, sink, recent, Br, Bc, stream=None) -> int:
+    """Direct call of the C entry point; returns its status code."""
+    return lib.ssa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(tile_skip_count),
+                       B, Hq, Hkv, Lq, Lk, d, int(causal), float(scale), int(mode), float(lam),
+                       int(n), int(m), int(sink), int(recent), Br, Bc, _stream(stream))
+
+
+def ssa_fwd_debug(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
+                  lam, n, m, sink, recent, Br, Bc, stream=None, skip_bits=None, keep_bits=None) -> int:
+    return lib.ssa_fwd_debug(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(tile_skip_count),
+                             B, Hq, Hkv, Lq, Lk, d, int(causal), float(scale), int(mode), float(lam),
+                             int(n), int(m), int(sink), int(recent), Br, Bc, _stream(stream),
+                             _ptr(skip_bits), _ptr(keep_bits))
+
+
+def attention(q, k, v, *, causal=True, scale=None, mode=MODE_SKIP, lam=0.0, n=0, m=0, sink=0,
+              recent=0, Br=128, Bc=128, stream=None, out=None, lse=None, counts=None,
+              skip_bits=None, keep_bits=None):
+    """Allocate outputs (torch) and run the forward through the C ABI.
+
+    q [B, Lq, Hq, d], k/v [B, Lk, Hkv, d] bf16 CUDA tensors.  Returns
+    (out [B, Lq, Hq, d] bf16, lse [B, Hq, Lq] fp32, tile_skip_count [B, Hq, nQ] int32).
+    """
+    B, Lq, Hq, d = q.shape
+    _, Lk, Hkv, _ = k.shape
+    if scale is None:
+        scale = d ** -0.5
+    nQ = -(-Lq // Br)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Hq, Lq, dtype=torch.float32, device=q.device)
+    if counts is None:
+        counts = torch.empty(B, Hq, nQ, dtype=torch.int32, device=q.device)
+    if skip_bits is None and keep_bits is None:
+        st = ssa_fwd(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode, lam,
+                     n, m, sink, recent, Br, Bc, stream)
+    else:
+        st = ssa_fwd_debug(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
+                           lam, n, m, sink, recent, Br, Bc, stream, skip_bits, keep_bits)
+    if st != SSA_OK:
+        raise SSAError(st, "ssa_fwd")
+    return out, lse, counts

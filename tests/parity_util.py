@@ -1,0 +1,123 @@
+"""Helpers for GPU-vs-oracle parity: run both sides on the same seeded bf16
+inputs and compare work item by work item.
+
+Bar (the method statement's tolerances): outputs max-abs <= 2e-2 and
+relative L2 <= 5e-3 against the fp64 oracle; lse max-abs <= 1e-3; skip
+decisions identical except tiles whose margin |exp(m_tile - m) - lambda| is
+below 1e-3 * lambda; N:M keep masks identical except keys whose fate is a
+near tie in fp32 (oracle tie bits: the two scores around the N-th place lie
+within 1e-4 * (1 + |s|) of each other, raw q.k units).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+from oracle import run_items
+
+OUT_MAX_ABS = 2e-2
+OUT_REL_L2 = 5e-3
+LSE_MAX_ABS = 1e-3
+TIE_TOL = 1e-4
+
+
+@dataclass
+class Report:
+    items: int = 0
+    out_max_abs: float = 0.0
+    out_rel_l2: float = 0.0
+    lse_max_abs: float = 0.0
+    skipped_gpu: int = 0
+    skipped_oracle: int = 0
+    visited: int = 0
+    marginal_mismatch: int = 0
+    keep_mismatch_ties: int = 0
+    notes: list = field(default_factory=list)
+
+
+def gpu_run(q, k, v, *, causal, scale, mode, lam=0.0, n=0, m=0, sink=0, recent=0, Br=128, Bc=128,
+            keep_bits=False):
+    from softmax_ssa_fwd_b200 import ssa
+    B, Lq, Hq, d = q.shape
+    Lk = k.shape[1]
+    nQ, nK = -(-Lq // Br), -(-Lk // Bc)
+    sb = torch.zeros(B, Hq, nQ, -(-nK // 32), dtype=torch.int32, device=q.device)
+    kb = torch.zeros(B, Hq, Lq, -(-Lk // 32), dtype=torch.int32, device=q.device) if keep_bits else None
+    out, lse, cnt = ssa.attention(q, k, v, causal=causal, scale=scale, mode=mode, lam=lam, n=n, m=m,
+                                  sink=sink, recent=recent, Br=Br, Bc=Bc, skip_bits=sb, keep_bits=kb)
+    st = ssa.ssa_device_status()
+    assert st == ssa.SSA_OK, ssa.status_string(st)
+    return out, lse, cnt, sb, kb
+
+
+def _unpack(words, nbits):
+    w = np.ascontiguousarray(words).view(np.uint32)
+    return np.unpackbits(w.view(np.uint8), axis=-1, bitorder="little")[..., :nbits].astype(bool)
+
+
+def compare(q, k, v, items, *, causal, scale, mode, lam=0.0, n=0, m=0, sink=0, recent=0, Br=128,
+            Bc=128, keep_bits=False, gpu=None, qkv_cpu=None) -> Report:
+    """Run (or reuse) the GPU result, run the oracle on ``items``, compare."""
+    if gpu is None:
+        gpu = gpu_run(q, k, v, causal=causal, scale=scale, mode=mode, lam=lam, n=n, m=m, sink=sink,
+                      recent=recent, Br=Br, Bc=Bc, keep_bits=keep_bits)
+    out, lse, cnt, sb, kb = gpu
+    qc, kc, vc = qkv_cpu if qkv_cpu is not None else (q.cpu(), k.cpu(), v.cpu())
+    B, Lq, Hq, d = qc.shape
+    Lk = kc.shape[1]
+    nK = -(-Lk // Bc)
+    res = run_items(qc, kc, vc, causal=causal, scale=scale, mode=mode, lam=lam, n=n, m=m, sink=sink,
+                    recent=recent, Br=Br, Bc=Bc, items=items, keep_bits=keep_bits, tie_tol=TIE_TOL)
+    rep = Report(items=len(items))
+    num = den = 0.0
+    for it, (b, h, t) in enumerate(res.items):
+        r0, r1 = t * Br, min(Lq, t * Br + Br)
+        rows = r1 - r0
+        g_sb = _unpack(sb[b, h, t].cpu().numpy(), nK)
+        o_sb = _unpack(res.skip_bits[it], nK)
+        marg = _unpack(res.marginal_bits[it], nK)
+        diff = g_sb != o_sb
+        assert not (diff & ~marg).any(), (
+            f"skip decision mismatch at item {(b, h, t)} tiles {np.nonzero(diff & ~marg)[0][:8]}")
+        rep.skipped_gpu += int(g_sb.sum())
+        rep.skipped_oracle += int(res.skip_count[it])
+        rep.visited += int(res.visited[it])
+        assert int(cnt[b, h, t]) == int(g_sb.sum())
+        if diff.any():
+            rep.marginal_mismatch += int(diff.sum())
+            rep.notes.append(f"item {(b, h, t)}: marginal decision differs, output not compared")
+            continue
+        assert int(cnt[b, h, t]) == int(res.skip_count[it])
+        if keep_bits:
+            g_kb = _unpack(kb[b, h, r0:r1].cpu().numpy(), Lk)
+            o_kb = _unpack(res.keep_bits[it, :rows], Lk)
+            ties = _unpack(res.tie_bits[it, :rows], Lk)
+            kd = g_kb != o_kb
+            assert not (kd & ~ties).any(), (
+                f"N:M keep mismatch at item {(b, h, t)}: {np.argwhere(kd & ~ties)[:8].tolist()}")
+            rep.keep_mismatch_ties += int(kd.sum())
+        go = out[b, r0:r1, h].float().cpu().numpy().astype(np.float64)
+        oo = res.out[it, :rows]
+        e = np.abs(go - oo)
+        rep.out_max_abs = max(rep.out_max_abs, float(e.max()))
+        num += float((e ** 2).sum())
+        den += float((oo ** 2).sum())
+        gl = lse[b, h, r0:r1].cpu().numpy().astype(np.float64)
+        ol = res.lse[it, :rows]
+        both_inf = np.isneginf(gl) & np.isneginf(ol)
+        assert (np.isneginf(gl) == np.isneginf(ol)).all()
+        if (~both_inf).any():
+            fin = ~both_inf
+            rep.lse_max_abs = max(rep.lse_max_abs, float(np.abs(gl[fin] - ol[fin]).max()))
+    rep.out_rel_l2 = (num / den) ** 0.5 if den > 0 else 0.0
+    assert rep.out_max_abs <= OUT_MAX_ABS, rep
+    assert rep.out_rel_l2 <= OUT_REL_L2, rep
+    assert rep.lse_max_abs <= LSE_MAX_ABS, rep
+    return rep
+
+
+def all_items(B, Hq, Lq, Br):
+    nQ = -(-Lq // Br)
+    return [(b, h, t) for b in range(B) for h in range(Hq) for t in range(nQ)]
