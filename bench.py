@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Bench: skip-softmax sparse attention forward on B200.
+
+Default workload: the Llama-3.1-8B-shaped prefill (B=1, Hq=32, Hkv=8,
+L=8192, d=128, causal, Br=Bc=128, skip-softmax lambda=1e-3), seeded
+synthetic bf16 Q/K/V.  One step = one ssa_fwd launch over that batch.
+
+Prints ONE JSON line.  ``value`` is the dense-equivalent attention TFLOP/s
+(4 d B Hq x visible pairs / time) summed over ranks; the same line carries
+executed TFLOP/s (2 Br Bc d x (visited + kept tiles) / time), the fraction of
+visited tiles skipped, tokens/s, the roofline of the kernel, an end-to-end
+figure through the C ABI with host buffers, and the CPU oracle's throughput on
+a bounded sample of the same workload.
+
+Multi-GPU: one process per GPU (torchrun); the path has no exchange step, so
+each rank runs its own replica of the workload (weak scaling) and time is the
+max over ranks.  ``--impl reference`` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from softmax_ssa_fwd_b200.inputs import MODE_NM, MODE_SKIP, WORKLOADS, make_inputs  # noqa: E402
+
+KERNEL_SRC = [os.path.join(ROOT, "softmax_ssa_fwd_b200", "csrc", f) for f in ("ssa_fwd.cu", "ptx.cuh")]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ssa_fwd_traffic.json")
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SRC:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d["bf16_tflops"], d.get("bf16_tflops_sustained"), d["hbm_gbs"], "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def dense_equiv_flops(w, Lq=None) -> float:
+    Lq = Lq or w.L
+    Lk = w.L
+    if w.causal:
+        off = Lk - Lq
+        i = np.arange(Lq, dtype=np.int64)
+        pairs = int(np.clip(i + off + 1, 0, Lk).sum())
+    else:
+        pairs = Lq * Lk
+    return 4.0 * w.d * w.B * w.Hq * pairs
+
+
+def workload_name(w, lam):
+    s = (f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} L={w.L} d={w.d} "
+         f"{'causal' if w.causal else 'non-causal'} Br={w.Br} Bc={w.Bc}")
+    if w.mode & MODE_SKIP:
+        s += f" skip lambda={lam:g}"
+    if w.mode & MODE_NM:
+        s += f" N:M {w.n}:{w.m} sink={w.sink} recent={w.recent}"
+    if w.sink_coef not in (0.0, 3.0) or w.local_alpha:
+        s += f" (stress: sink_coef={w.sink_coef:g} local_alpha={w.local_alpha:g})"
+    return s
+
+
+class Clocks:
+    """nvidia-smi sampler running during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        ids = [x for x in vis.split(",") if x.strip()] if vis else []
+        self.idx = ids[local_rank].strip() if local_rank < len(ids) else local_rank
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        rows_by_gpu = {}
+        for line in self.out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows_by_gpu.setdefault(parts[0], []).append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        rows = rows_by_gpu.get(str(self.idx))
+        if rows is None and len(rows_by_gpu) == 1:
+            rows = next(iter(rows_by_gpu.values()))
+        rows = rows or []
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        maxmhz = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[0] > 0.3 * maxmhz] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": maxmhz,
+                "reasons": reasons, "samples": len(loaded)}
+
+
+_CPU_INPUTS = {}
+
+
+def cpu_baseline(w, lam, budget_s: float, seed: int = 7):
+    """Time the fp64 oracle on a bounded random sample of work items of the
+    same workload (inputs generated on the CPU with the same recipe)."""
+    from oracle import run_items
+    g = torch.Generator().manual_seed(seed)
+    if w not in _CPU_INPUTS:
+        _CPU_INPUTS[w] = make_inputs(w, "cpu")
+    q, k, v = _CPU_INPUTS[w]
+    cores = len(os.sched_getaffinity(0))
+    nQ = -(-w.L // w.Br)
+    done_items, flops, t_total = 0, 0.0, 0.0
+    while done_items == 0 or t_total < budget_s:
+        n = cores
+        items = [(int(torch.randint(w.B, (1,), generator=g)), int(torch.randint(w.Hq, (1,), generator=g)),
+                  int(torch.randint(nQ, (1,), generator=g))) for _ in range(n)]
+        t0 = time.perf_counter()
+        run_items(q, k, v, causal=w.causal, scale=w.scale, mode=w.mode, lam=lam, n=w.n, m=w.m,
+                  sink=w.sink, recent=w.recent, Br=w.Br, Bc=w.Bc, items=items, nthreads=cores)
+        t_total += time.perf_counter() - t0
+        for (_, _, t) in items:
+            r0, r1 = t * w.Br, min(w.L, t * w.Br + w.Br)
+            if w.causal:
+                flops += 4.0 * w.d * sum(min(i + 1, w.L) for i in range(r0, r1))
+            else:
+                flops += 4.0 * w.d * (r1 - r0) * w.L
+        done_items += n
+    return {"value": flops / t_total / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done_items} random (b, head, q-tile) work items of {w.name} (lambda={lam:g}), "
+                      f"fp64 C oracle, {t_total:.1f} s wall; dense-equivalent FLOPs of the sample / wall"}
+
+
+def run_reference(args, w, lam, rank, world):
+    if rank != 0:
+        return 0
+    # each step: one batch of work items (one per host core) of the workload
+    per_step = []
+    info = None
+    for s in range(min(args.warmup, 1)):
+        cpu_baseline(w, lam, 0.0, seed=99)
+    for s in range(max(1, args.steps)):
+        info = cpu_baseline(w, lam, 0.0, seed=100 + s)
+        per_step.append(info["value"])
+    val = statistics.median(per_step)
+    line = {"impl": "reference", "metric": "attn fwd TFLOP/s (dense-equiv)", "value": val,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": workload_name(w, lam)},
+            "cpu_baseline": dict(info, value=val),
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama8k", choices=sorted(WORKLOADS))
+    ap.add_argument("--lam", type=float, default=None)
+    ap.add_argument("--sink-coef", type=float, default=None)
+    ap.add_argument("--local-alpha", type=float, default=None)
+    ap.add_argument("--L", type=int, default=None, help="override the sequence length")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+
+    w = WORKLOADS[args.workload]
+    if args.sink_coef is not None:
+        w = w.with_(sink_coef=args.sink_coef)
+    if args.local_alpha is not None:
+        w = w.with_(local_alpha=args.local_alpha)
+    if args.L is not None:
+        if w.rope == "3d":
+            raise SystemExit("--L does not apply to the 3D-rotary video workload")
+        w = w.with_(L=args.L, name=f"{w.name}@L{args.L}")
+    lam = args.lam if args.lam is not None else (1e-3 if w.mode & MODE_SKIP else 0.0)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, w, lam, rank, world)
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from softmax_ssa_fwd_b200 import ssa
+
+    dev = torch.device("cuda", local_rank)
+    # two input sets, alternated between steps: 2 x 168 MB > 126 MB L2
+    sets = []
+    for s in range(2):
+        q, k, v = make_inputs(w.with_(seed=w.seed + 1000 * s + 17 * rank), dev)
+        out = torch.empty_like(q)
+        lse = torch.empty(w.B, w.Hq, w.L, dtype=torch.float32, device=dev)
+        cnt = torch.empty(w.B, w.Hq, -(-w.L // w.Br), dtype=torch.int32, device=dev)
+        sets.append((q, k, v, out, lse, cnt))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        q, k, v, out, lse, cnt = sets[i & 1]
+        st = ssa.ssa_fwd(q, k, v, out, lse, cnt, w.B, w.Hq, w.Hkv, w.L, w.L, w.d, w.causal, w.scale,
+                         w.mode, lam, w.n, w.m, w.sink, w.recent, w.Br, w.Bc, stream)
+        if st != 0:
+            raise RuntimeError(ssa.status_string(st))
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if ssa.ssa_device_status(stream) != 0:
+        raise RuntimeError("device-side timeout during warm-up")
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        e1.synchronize()
+        torch.cuda.synchronize()
+        barrier()
+    ms = e0.elapsed_time(e1)
+    if ssa.ssa_device_status(stream) != 0:
+        raise RuntimeError("device-side timeout in the timed region")
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+
+    # skip statistics of the timed workload (identical every step per input set)
+    visited = ssa.ssa_visited_tiles(w.causal, w.L, w.L, w.Br, w.Bc) * w.B * w.Hq
+    skipped = sum(int(s[5].sum()) for s in sets) / len(sets)
+    kept = visited - skipped
+    flops_dense = dense_equiv_flops(w)
+    flops_exec = 2.0 * w.Br * w.Bc * w.d * (visited + kept)
+    tflops_dense = world * flops_dense / (ms_step * 1e-3) / 1e12
+    tflops_exec = world * flops_exec / (ms_step * 1e-3) / 1e12
+    bf16_peak, bf16_sus, hbm_peak, src = peaks()
+    tokens = world * w.B * w.L / (ms_step * 1e-3)
+
+    traffic = None
+    if os.path.exists(TRAFFIC_FILE):
+        with open(TRAFFIC_FILE) as f:
+            tr = json.load(f)
+        if tr.get("kernel_hash") == kernel_hash() and tr.get("workload") == w.name:
+            traffic = tr.get("dram_bytes_per_launch")
+
+    # end to end through the C ABI with host buffers: pinned host inputs ->
+    # device, forward, out + lse + counts back to pinned host, every step
+    e2e = None
+    if not args.no_e2e:
+        q, k, v, out, lse, cnt = sets[0]
+        hq_, hk_, hv_ = (t.cpu().pin_memory() for t in (q, k, v))
+        ho, hl, hc = (torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (out, lse, cnt))
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hc))
+        n_e2e = max(3, min(args.steps, 30))
+
+        def e2e_step():
+            dq.copy_(hq_, non_blocking=True)
+            dk.copy_(hk_, non_blocking=True)
+            dv.copy_(hv_, non_blocking=True)
+            st = ssa.ssa_fwd(dq, dk, dv, out, lse, cnt, w.B, w.Hq, w.Hkv, w.L, w.L, w.d, w.causal,
+                             w.scale, w.mode, lam, w.n, w.m, w.sink, w.recent, w.Br, w.Bc, stream)
+            if st != 0:
+                raise RuntimeError(ssa.status_string(st))
+            ho.copy_(out, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+            hc.copy_(cnt, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        e1.synchronize()
+        barrier()
+        ems = e0.elapsed_time(e1)
+        if dist is not None:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * flops_dense / (ems / n_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems / n_e2e,
+               "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, lam, args.cpu_budget)
+
+    if rank == 0:
+        clocks = clk.summary()
+        line = {
+            "metric": "attn fwd TFLOP/s (dense-equiv)",
+            "value": tflops_dense, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload_name(w, lam), "parallelism": f"replicas x{world}",
+                       "l2": "inputs alternate between 2 sets of 168 MB each (> 126 MB L2)"},
+            "executed_tflops": tflops_exec,
+            "executed_frac_of_peak": tflops_exec / world / bf16_peak,
+            "tiles_skipped_frac": skipped / visited,
+            "tiles_visited": visited, "tiles_skipped": skipped,
+            "tokens_per_s": tokens,
+            "roofline": {"bound": "tensor", "achieved": flops_exec / (ms_step * 1e-3) / 1e12,
+                         "peak": bf16_peak, "unit": "TFLOP/s",
+                         "frac": flops_exec / (ms_step * 1e-3) / 1e12 / bf16_peak,
+                         "traffic": traffic, "peak_source": f"{src} bf16 burst",
+                         "kernel": "ssa::ssa_fwd_kernel<128,128>",
+                         "dense_equiv_frac": flops_dense / (ms_step * 1e-3) / 1e12 / bf16_peak,
+                         "hbm_frac_of_algorithmic_bytes": None},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "kernel_hash": kernel_hash(),
+        }
+        alg_bytes = 2 * (2 * w.B * w.L * w.Hq * w.d + 2 * w.B * w.L * w.Hkv * w.d) + 4 * w.B * w.Hq * w.L
+        line["roofline"]["hbm_frac_of_algorithmic_bytes"] = alg_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

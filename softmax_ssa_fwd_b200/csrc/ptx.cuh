@@ -167,6 +167,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       SSA_W8(0), SSA_W8(8), SSA_W8(16), SSA_W8(24)
       : "memory");
 }
+#define SSA_F8(i) "=f"(r[i + 0]), "=f"(r[i + 1]), "=f"(r[i + 2]), "=f"(r[i + 3]), \
+                  "=f"(r[i + 4]), "=f"(r[i + 5]), "=f"(r[i + 6]), "=f"(r[i + 7])
+// Same as tmem_ld32, straight into fp32 registers (no copies after the load).
+__device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : SSA_F8(0), SSA_F8(8), SSA_F8(16), SSA_F8(24)
+      : "r"(taddr));
+}
+#undef SSA_F8
 #undef SSA_R8
 #undef SSA_W8
 

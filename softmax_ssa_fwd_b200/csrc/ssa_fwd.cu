@@ -10,23 +10,29 @@
 //   custom N:M configuration): per M consecutive keys keep the top-N scores,
 //   the rest become -inf; sink and recent-window keys stay dense.
 //
-// One CTA owns 128 query rows of one (batch, query head) and walks the key
-// tiles it can see.  Warp roles (256 threads):
+// One CTA owns two 128-row query tiles (A and B, adjacent in the sequence) of
+// one (batch, query head) and walks the key tiles they can see; K and V tiles
+// are loaded once for both.  Warp roles (384 threads):
 //   warp 0      Q and K producer: TMA into a KST-deep K ring
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T and O += P V on tcgen05
-//   warp 2      V producer: issues a V tile's TMA only after the tile's keep
-//               decision, so a skipped tile never loads V
-//   warps 4..7  softmax: thread t owns query row t (TMEM lane t); masks, N:M
-//               top-N in registers, tile row max, skip vote, exp2, P -> TMEM,
-//               lazy O rescale, epilogue
-// TMEM (512 columns): S/P double buffer at columns 0 and 128, O at 256.
-// P (bf16, two per 32-bit column) overwrites the S buffer it came from and is
-// the A operand of the P.V MMA straight from TMEM.
+//   warp 1      TMEM owner and MMA issuer: S_t = Q_t K^T and O_t += P_t V on
+//               tcgen05, ping-ponging between the two tiles so the tensor pipe
+//               works on one tile while the other tile's softmax runs
+//   warp 2      V producer: issues a V tile's TMA only once a tile has decided
+//               to keep it, so a tile skipped by both never loads V
+//   warps 4..7  softmax of tile A, warps 8..11 softmax of tile B: thread r
+//               owns query row r (TMEM lane r): masks, N:M top-N in registers,
+//               tile row max, skip vote, exp2, P -> TMEM, lazy O rescale,
+//               epilogue
+// TMEM (512 columns): tile t uses S/P at column 256 t and O at 256 t + 128.
+// P (bf16, two per 32-bit column) overwrites the S columns it came from and
+// is the A operand of the P.V MMA straight from TMEM.  Because S_t(j+1) is
+// issued after O_t += P_t(j) V_j, the completion of S_t(j+1) also proves
+// that every earlier P.V of tile t has finished, so the softmax may rescale
+// O_t without another wait.
 //
-// When Br = 64 the 128-row CTA tile carries two logical query tiles (rows
-// 0-63 and 64-127) that vote, count and keep state separately; a V tile is
-// loaded and P.V issued when either keeps the key tile, with P = 0 for the
-// half that skipped.
+// When Br = 64 each 128-row tile carries two logical query tiles (rows 0-63
+// and 64-127) that vote, count and keep state separately; P.V is issued when
+// either keeps the key tile, with P = 0 for the half that skipped.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -41,15 +47,16 @@
 
 namespace ssa {
 
-constexpr int BM = 128;       // CTA query rows = tcgen05 M
-constexpr int KST = 3;        // K ring depth
+constexpr int BM = 128;       // rows per query tile = tcgen05 M
+constexpr int NQT = 2;        // query tiles per CTA
+constexpr int KST = 2;        // K ring depth
 constexpr int VST = 2;        // V ring depth
-constexpr int NTHREADS = 256;
+constexpr int NTHREADS = 384;
 constexpr int TMEM_COLS = 512;
-constexpr int S_COL = 0;      // S/P buffer b at column S_COL + 128 * b
-constexpr int O_COL = 256;
 constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;  // 2 s per wait
 constexpr float RESCALE_LOG2 = 8.0f;  // lazy O rescale once the max grew by 2^8
+// One exp2 in POLY_EVERY pairs runs as a polynomial on the FMA pipe.
+constexpr int POLY_EVERY = 4;
 
 struct Params {
   __nv_bfloat16* out;
@@ -60,8 +67,7 @@ struct Params {
   int* status;
   int B, Hq, Hkv, Lq, Lk, causal, mode, n, m, sink, recent;
   int half;   // Br == 64
-  int Br;
-  int nQp;    // 128-row CTA tiles per (b, hq)
+  int nQp;    // 128-row tiles per (b, hq)
   int nQ;     // logical query tiles per (b, hq)
   int nK;     // key tiles
   int nKw;    // words of skip bits per logical query tile
@@ -75,21 +81,20 @@ struct __align__(8) Bars {
   uint64_t q_full;
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
-  uint64_t s_full[2], dec_ready[2], p_ready[2];
-  uint64_t o_bar, o_final;
+  uint64_t s_full[NQT], dec_ready[NQT], dec_ack[NQT], p_ready[NQT], o_done[NQT];
   uint32_t tmem_base;
-  uint32_t dec_word[2];
-  uint32_t vote[2][4];
+  uint32_t dec_word[NQT];
+  uint32_t vote[NQT][2][4];
   uint32_t abort_flag;
 };
 
 template <int D, int BC>
 struct Smem {
-  static constexpr uint32_t Q_BYTES = BM * D * 2;
+  static constexpr uint32_t QT_BYTES = BM * D * 2;  // one query tile
   static constexpr uint32_t K_BYTES = BC * D * 2;
   static constexpr uint32_t V_BYTES = BC * D * 2;
   static constexpr uint32_t Q_OFF = 0;
-  static constexpr uint32_t K_OFF = Q_OFF + Q_BYTES;
+  static constexpr uint32_t K_OFF = Q_OFF + NQT * QT_BYTES;
   static constexpr uint32_t V_OFF = K_OFF + KST * K_BYTES;
   static constexpr uint32_t BAR_OFF = V_OFF + VST * V_BYTES;
   static constexpr uint32_t TOTAL = BAR_OFF + ((sizeof(Bars) + 127) / 128) * 128;
@@ -110,10 +115,32 @@ __host__ __device__ inline int visited_key_tiles(int causal, int Lq, int Lk, int
   return t > nK ? nK : (int)t;
 }
 
-__device__ __forceinline__ float fast_exp2(float x) {
+__device__ __forceinline__ float mufu_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe: x = n + f with n = rint(x) (by the 1.5 * 2^23 shift),
+// f in [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial (max relative error
+// 7.5e-5, below bf16 resolution; coefficients from csrc/fit_exp2_poly.py);
+// 2^n by adding n to the exponent field.  Arguments below -126 give 0.
+__device__ __forceinline__ float2 poly_exp2x2(float x0, float x1) {
+  constexpr float SHIFT = 12582912.0f;  // 1.5 * 2^23
+  constexpr float C0 = 0x1.fff692p-1f, C1 = 0x1.62f31ap-1f, C2 = 0x1.f0de1ap-3f, C3 = 0x1.c3f76p-5f;
+  const float a0 = fmaxf(x0, -127.f), a1 = fmaxf(x1, -127.f);
+  float r0, r1, f0, f1, p0, p1;
+  asm("add.rn.f32 %0, %1, %2;" : "=f"(r0) : "f"(a0), "f"(SHIFT));
+  asm("add.rn.f32 %0, %1, %2;" : "=f"(r1) : "f"(a1), "f"(SHIFT));
+  asm("sub.rn.f32 %0, %1, %2;" : "=f"(f0) : "f"(r0), "f"(SHIFT));
+  asm("sub.rn.f32 %0, %1, %2;" : "=f"(f1) : "f"(r1), "f"(SHIFT));
+  f0 = a0 - f0;
+  f1 = a1 - f1;
+  p0 = fmaf(fmaf(fmaf(C3, f0, C2), f0, C1), f0, C0);
+  p1 = fmaf(fmaf(fmaf(C3, f1, C2), f1, C1), f1, C0);
+  const uint32_t b0 = __float_as_uint(p0) + (__float_as_uint(r0) << 23);
+  const uint32_t b1 = __float_as_uint(p1) + (__float_as_uint(r1) << 23);
+  return make_float2(x0 < -126.f ? 0.f : __uint_as_float(b0), x1 < -126.f ? 0.f : __uint_as_float(b1));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -129,10 +156,19 @@ __device__ __forceinline__ bool aborted(Bars* bars) {
   return *reinterpret_cast<volatile uint32_t*>(&bars->abort_flag) != 0u;
 }
 
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // N:M selection on one thread's row: for each aligned group of M keys keep a
-// key iff it is visible and (inside the sink / recent window, or among the N
-// largest scores of its group, equal scores ranked by lower index).  Dropped
-// keys become -inf.  Returns a bit per column of the BC-wide tile.
+// key iff (inside the sink / recent window, or among the N largest scores of
+// its group, equal scores ranked by lower index); dropped keys become -inf.
+// Masked keys are already -inf, rank last and stay -inf.
 template <int M, int BC>
 __device__ __forceinline__ void nm_select(float (&x)[BC], int N, int col0, int pos, int sink,
                                           int recent) {
@@ -158,7 +194,256 @@ __device__ __forceinline__ void nm_select(float (&x)[BC], int N, int col0, int p
   }
 }
 
-template <int D, int BC>
+struct Work {
+  int b, hq, hkv;
+  int pt[NQT];            // 128-row tile index of tile t
+  int nvis_h[NQT][2];     // visited key tiles per logical half
+  int nvis_t[NQT];        // per tile
+  int nvis;               // per CTA
+};
+
+template <int D, int BC, int NM_M, bool DBG>
+__device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b, int hq, int t,
+                                             int pt, int nvis_h0, int nvis_h1, uint32_t tmem) {
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int row = tid - 128 - 128 * t;
+  const int quarter = warp & 3;
+  const int half = p.half ? (row >> 6) : 0;
+  const int grow = pt * BM + row;
+  const bool valid = grow < p.Lq;
+  const int pos = grow + p.Lk - p.Lq;
+  const int pos_first = pt * BM + p.Lk - p.Lq;
+  const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
+  const uint32_t s_col = 256 * t, o_col = 256 * t + 128;
+  const bool skip_on = (p.mode & SSA_MODE_SKIP) != 0;
+  constexpr bool nm_on = NM_M != 0;
+  const bool leader = p.half ? ((row & 63) == 0) : (row == 0);
+  const int my_nvis = half ? nvis_h1 : nvis_h0;
+  const int nvis = nvis_h0 > nvis_h1 ? nvis_h0 : nvis_h1;
+  const uint32_t bar_vote = 1 + t, bar_p = 3 + t;
+
+  float m_true = -INFINITY;  // running max over kept tiles (raw q.k units)
+  float m_ref = -INFINITY;   // reference the O accumulator and l are scaled to
+  float l = 0.f;
+  int n_pv = 0;
+  int skipped = 0;
+  uint32_t skip_word = 0;
+  bool failed = false;
+
+  for (int j = 0; j < nvis; ++j) {
+    bool ok = !failed && mbar_wait(smem_u32(&bars->s_full[t]), j & 1, WAIT_TIMEOUT_NS);
+    ok = __all_sync(0xffffffffu, ok);
+    float m_tile = -INFINITY;
+    const int col0 = j * BC;
+    // Pass 1, 64 columns at a time: masks, N:M, tile row max.  Masked
+    // scores are written back to TMEM so pass 2 needs no mask.
+    const bool need_mask = (col0 + BC > p.Lk) || (p.causal && col0 + BC - 1 > pos_first);
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int bb = 0; bb < BC / 64; ++bb) {
+        float x[64];
+        const uint32_t ta = lane_base + s_col + 64 * bb;
+        tmem_ld32f(ta, &x[0]);
+        tmem_ld32f(ta + 32, &x[32]);
+        tmem_wait_ld();
+        const int cb = col0 + 64 * bb;
+        if (need_mask) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const int jj = cb + i;
+            if (jj >= p.Lk || (p.causal && jj > pos)) x[i] = -INFINITY;
+          }
+        }
+        if constexpr (nm_on) nm_select<(NM_M ? NM_M : 4), 64>(x, p.n, cb, pos, p.sink, p.recent);
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 64; i += 4) {
+          mx0 = fmaxf(mx0, fmaxf(x[i], x[i + 1]));
+          mx1 = fmaxf(mx1, fmaxf(x[i + 2], x[i + 3]));
+        }
+        m_tile = fmaxf(m_tile, fmaxf(mx0, mx1));
+        if (need_mask || nm_on) {
+          tmem_st32(ta, *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
+          tmem_st32(ta + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));
+        }
+        if (DBG && p.keep_bits != nullptr && valid && j < my_nvis) {
+          uint32_t* kb = p.keep_bits + ((size_t)(b * p.Hq + hq) * p.Lq + grow) * p.Lkw;
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) word |= (x[32 * w + u] != -INFINITY ? 1u : 0u) << u;
+            const int wi = cb / 32 + w;
+            if (wi < p.Lkw) kb[wi] = word;
+          }
+        }
+      }
+      if (need_mask || nm_on) tmem_wait_st();
+    }
+    const bool negligible =
+        !valid || m_tile == -INFINITY ||
+        (m_true != -INFINITY && (m_tile - m_true) * p.scale_log2 < p.log2_lambda);
+    const uint32_t wneg = __all_sync(0xffffffffu, negligible) ? 1u : 0u;
+    if (lane == 0) bars->vote[t][j & 1][quarter] = wneg | (ok ? 0u : 2u);
+    tc_fence_before();
+    named_bar_sync(bar_vote, 128);
+    uint32_t v4[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) v4[w] = *reinterpret_cast<volatile uint32_t*>(&bars->vote[t][j & 1][w]);
+    if ((v4[0] | v4[1] | v4[2] | v4[3]) & 2u) {
+      failed = true;
+      if (row == 0) record_failure(p, bars);
+      break;
+    }
+    bool keep_h[2];
+    if (p.half) {
+      keep_h[0] = (j < nvis_h0) && !(skip_on && (v4[0] & v4[1] & 1u));
+      keep_h[1] = (j < nvis_h1) && !(skip_on && (v4[2] & v4[3] & 1u));
+    } else {
+      keep_h[0] = keep_h[1] = !(skip_on && (v4[0] & v4[1] & v4[2] & v4[3] & 1u));
+    }
+    const bool tile_keep = keep_h[0] || keep_h[1];
+    const bool my_keep = half ? keep_h[1] : keep_h[0];
+    if (leader && j < my_nvis) {
+      if (!my_keep) {
+        ++skipped;
+        skip_word |= 1u << (j & 31);
+      }
+      if (DBG && p.skip_bits != nullptr && ((j & 31) == 31 || j == my_nvis - 1)) {
+        const int qt = p.half ? 2 * pt + half : pt;
+        p.skip_bits[((size_t)(b * p.Hq + hq) * p.nQ + qt) * p.nKw + (j >> 5)] = skip_word;
+        skip_word = 0;
+      }
+    }
+    if (row == 0) {
+      // the V producer must have taken decision j-1 before decision j is
+      // published on the same barrier (keeps its phases from aliasing)
+      if (j > 0 && !mbar_wait(smem_u32(&bars->dec_ack[t]), (j - 1) & 1, WAIT_TIMEOUT_NS))
+        record_failure(p, bars);
+      bars->dec_word[t] = tile_keep ? 1u : 0u;
+      mbar_arrive(smem_u32(&bars->dec_ready[t]));
+      if (!tile_keep) mbar_arrive(smem_u32(&bars->p_ready[t]));
+    }
+    if (!tile_keep) continue;
+
+    if (my_keep) {
+      m_true = fmaxf(m_true, m_tile);
+      bool resc = false;
+      if (m_ref == -INFINITY) m_ref = m_true;  // first kept key: O and l are still zero
+      else resc = (m_true - m_ref) * p.scale_log2 > RESCALE_LOG2;
+      if (__any_sync(0xffffffffu, resc)) {
+        // every earlier P.V of this tile completed before S(j) did
+        const float alpha = resc ? mufu_exp2((m_ref - m_true) * p.scale_log2) : 1.f;
+        if (n_pv > 0) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + o_col + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(lane_base + o_col + 32 * c, o);
+          }
+        }
+        if (resc) {
+          l *= alpha;
+          m_ref = m_true;
+        }
+      }
+      // Pass 2: P = exp2((s - m_ref) * scale * log2 e), 64 columns at a time
+      const float c = p.scale_log2;
+      const float mref_s = (m_ref == -INFINITY) ? 0.f : m_ref * c;
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int bb = 0; bb < BC / 64; ++bb) {
+        float x[64];
+        const uint32_t ta = lane_base + s_col + 64 * bb;
+        tmem_ld32f(ta, &x[0]);
+        tmem_ld32f(ta + 32, &x[32]);
+        tmem_wait_ld();
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float a0 = fmaf(x[2 * i], c, -mref_s);
+          const float a1 = fmaf(x[2 * i + 1], c, -mref_s);
+          float p0, p1;
+          if ((i % POLY_EVERY) == POLY_EVERY - 1) {
+            const float2 ev = poly_exp2x2(a0, a1);
+            p0 = ev.x;
+            p1 = ev.y;
+          } else {
+            p0 = mufu_exp2(a0);
+            p1 = mufu_exp2(a1);
+          }
+          ls0 += p0;
+          ls1 += p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(lane_base + s_col + 32 * bb, pk);
+      }
+      l += ls0 + ls1;
+    } else {
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) pk[i] = 0u;
+#pragma unroll
+      for (int h = 0; h < BC / 64; ++h) tmem_st32(lane_base + s_col + 32 * h, pk);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    named_bar_sync(bar_p, 128);
+    if (row == 0) mbar_arrive(smem_u32(&bars->p_ready[t]));
+    ++n_pv;
+  }
+
+  // ---- epilogue
+  bool okf = true;
+  if (nvis > 0) okf = mbar_wait(smem_u32(&bars->o_done[t]), 0, WAIT_TIMEOUT_NS);
+  if (!okf) record_failure(p, bars);
+  okf = __all_sync(0xffffffffu, okf) && !failed;
+  tc_fence_after();
+  const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+  __nv_bfloat16* orow = p.out + ((size_t)(b * p.Lq + grow) * p.Hq + hq) * D;
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t o[32];
+    if (okf && n_pv > 0) {
+      tmem_ld32(lane_base + o_col + 32 * c, o);
+      tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = 0u;
+    }
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+      for (int v8 = 0; v8 < 4; ++v8) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(o[8 * v8 + 0]) * inv_l, __uint_as_float(o[8 * v8 + 1]) * inv_l);
+        w.y = pack_bf16x2(__uint_as_float(o[8 * v8 + 2]) * inv_l, __uint_as_float(o[8 * v8 + 3]) * inv_l);
+        w.z = pack_bf16x2(__uint_as_float(o[8 * v8 + 4]) * inv_l, __uint_as_float(o[8 * v8 + 5]) * inv_l);
+        w.w = pack_bf16x2(__uint_as_float(o[8 * v8 + 6]) * inv_l, __uint_as_float(o[8 * v8 + 7]) * inv_l);
+        dst[v8] = w;
+      }
+    }
+  }
+  if (valid)
+    p.lse[(size_t)(b * p.Hq + hq) * p.Lq + grow] = (l > 0.f) ? m_ref * p.scale + logf(l) : -INFINITY;
+  if (leader) {
+    const int qt = p.half ? 2 * pt + half : pt;
+    if (qt < p.nQ) {
+      p.skip_count[(size_t)(b * p.Hq + hq) * p.nQ + qt] = skipped;
+      if (p.skip_bits != nullptr) {
+        uint32_t* sb = p.skip_bits + ((size_t)(b * p.Hq + hq) * p.nQ + qt) * p.nKw;
+        for (int w = (my_nvis + 31) / 32; w < p.nKw; ++w) sb[w] = 0u;
+      }
+    }
+  }
+}
+
+template <int D, int BC, int NM_M, bool DBG>
 __global__ void __launch_bounds__(NTHREADS, 1)
     ssa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -173,23 +458,36 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // ---- work item: heaviest causal tiles first; query heads that share a KV
+  // ---- work item: heaviest causal pairs first; query heads that share a KV
   // head are adjacent in launch order.
-  const int per_tile = p.B * p.Hq;
-  int pt = blockIdx.x / per_tile;
-  if (p.causal) pt = p.nQp - 1 - pt;
-  const int bh = blockIdx.x % per_tile;
-  const int b = bh / p.Hq, hq = bh % p.Hq;
-  const int hkv = hq / (p.Hq / p.Hkv);
-
-  int nvis_h[2];
-  if (p.half) {
-    nvis_h[0] = (2 * pt < p.nQ) ? visited_key_tiles(p.causal, p.Lq, p.Lk, 64, BC, 2 * pt) : 0;
-    nvis_h[1] = (2 * pt + 1 < p.nQ) ? visited_key_tiles(p.causal, p.Lq, p.Lk, 64, BC, 2 * pt + 1) : 0;
-  } else {
-    nvis_h[0] = nvis_h[1] = visited_key_tiles(p.causal, p.Lq, p.Lk, BM, BC, pt);
+  Work wk;
+  {
+    const int per_pair = p.B * p.Hq;
+    const int npairs = (p.nQp + 1) / 2;
+    int pair = blockIdx.x / per_pair;
+    if (p.causal) pair = npairs - 1 - pair;
+    const int bh = blockIdx.x % per_pair;
+    wk.b = bh / p.Hq;
+    wk.hq = bh % p.Hq;
+    wk.hkv = wk.hq / (p.Hq / p.Hkv);
+    wk.nvis = 0;
+#pragma unroll
+    for (int t = 0; t < NQT; ++t) {
+      const int pt = 2 * pair + t;
+      wk.pt[t] = pt;
+      if (pt >= p.nQp) {
+        wk.nvis_h[t][0] = wk.nvis_h[t][1] = 0;
+      } else if (p.half) {
+        wk.nvis_h[t][0] = (2 * pt < p.nQ) ? visited_key_tiles(p.causal, p.Lq, p.Lk, 64, BC, 2 * pt) : 0;
+        wk.nvis_h[t][1] = (2 * pt + 1 < p.nQ) ? visited_key_tiles(p.causal, p.Lq, p.Lk, 64, BC, 2 * pt + 1) : 0;
+      } else {
+        wk.nvis_h[t][0] = wk.nvis_h[t][1] = visited_key_tiles(p.causal, p.Lq, p.Lk, BM, BC, pt);
+      }
+      wk.nvis_t[t] = wk.nvis_h[t][0] > wk.nvis_h[t][1] ? wk.nvis_h[t][0] : wk.nvis_h[t][1];
+      if (wk.nvis_t[t] > wk.nvis) wk.nvis = wk.nvis_t[t];
+    }
   }
-  const int nvis = nvis_h[0] > nvis_h[1] ? nvis_h[0] : nvis_h[1];
+  const int nvis = wk.nvis;
 
   // ---- set-up
   if (tid == 0) {
@@ -202,13 +500,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(smem_u32(&bars->v_full[i]), 1);
       mbar_init(smem_u32(&bars->v_empty[i]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NQT; ++i) {
       mbar_init(smem_u32(&bars->s_full[i]), 1);
       mbar_init(smem_u32(&bars->dec_ready[i]), 1);
+      mbar_init(smem_u32(&bars->dec_ack[i]), 1);
       mbar_init(smem_u32(&bars->p_ready[i]), 1);
+      mbar_init(smem_u32(&bars->o_done[i]), 1);
     }
-    mbar_init(smem_u32(&bars->o_bar), 1);
-    mbar_init(smem_u32(&bars->o_final), 1);
     bars->abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -225,14 +523,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 0) {
-    // ======================= Q / K producer =======================
-    if (lane == 0 && nvis > 0) {
+  if (warp < 4) {
+    reg_dealloc<104>();
+    if (warp == 0 && lane == 0 && nvis > 0) {
+      // ======================= Q / K producer =======================
       const uint32_t qbar = smem_u32(&bars->q_full);
-      mbar_arrive_expect_tx(qbar, L::Q_BYTES);
+      uint32_t qbytes = 0;
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c)
-        tma_load_4d(q_s + c * BM * 128, &tm_q, qbar, c * 64, hq, pt * BM, b);
+      for (int t = 0; t < NQT; ++t)
+        if (wk.nvis_t[t] > 0) qbytes += L::QT_BYTES;
+      mbar_arrive_expect_tx(qbar, qbytes);
+#pragma unroll
+      for (int t = 0; t < NQT; ++t)
+        if (wk.nvis_t[t] > 0)
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(q_s + t * L::QT_BYTES + c * BM * 128, &tm_q, qbar, c * 64, wk.hq, wk.pt[t] * BM, wk.b);
       int issued = 0;
       for (int j = 0; j < nvis; ++j) {
         const int slot = j % KST;
@@ -245,305 +551,148 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive_expect_tx(fb, L::K_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(k_s + slot * L::K_BYTES + c * BC * 128, &tm_k, fb, c * 64, hkv, j * BC, b);
+          tma_load_4d(k_s + slot * L::K_BYTES + c * BC * 128, &tm_k, fb, c * 64, wk.hkv, j * BC, wk.b);
         issued = j + 1;
       }
       // drain: the newest load of each slot (older ones were consumed)
-      mbar_wait(qbar, 0, WAIT_TIMEOUT_NS);
+      bool drained = mbar_wait(qbar, 0, WAIT_TIMEOUT_NS);
       for (int j = issued - KST; j < issued; ++j)
-        if (j >= 0) mbar_wait(smem_u32(&bars->k_full[j % KST]), (j / KST) & 1, WAIT_TIMEOUT_NS);
-    }
-  } else if (warp == 2) {
-    // ======================= V producer =======================
-    if (lane == 0) {
+        if (j >= 0) drained &= mbar_wait(smem_u32(&bars->k_full[j % KST]), (j / KST) & 1, WAIT_TIMEOUT_NS);
+      if (!drained) record_failure(p, bars);
+    } else if (warp == 2 && lane == 0) {
+      // ======================= V producer =======================
       int last_load[VST];
       for (int i = 0; i < VST; ++i) last_load[i] = -1;
       for (int j = 0; j < nvis; ++j) {
         if (aborted(bars)) break;
-        if (!mbar_wait(smem_u32(&bars->dec_ready[j & 1]), (j >> 1) & 1, WAIT_TIMEOUT_NS)) {
-          record_failure(p, bars);
-          break;
-        }
-        const uint32_t keep = *reinterpret_cast<volatile uint32_t*>(&bars->dec_word[j & 1]);
         const int slot = j % VST;
         if (!mbar_wait(smem_u32(&bars->v_empty[slot]), ((j / VST) & 1) ^ 1, WAIT_TIMEOUT_NS)) {
           record_failure(p, bars);
           break;
         }
         const uint32_t fb = smem_u32(&bars->v_full[slot]);
-        if (keep) {
-          mbar_arrive_expect_tx(fb, L::V_BYTES);
+        bool loaded = false, fail = false;
 #pragma unroll
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_4d(v_s + slot * L::V_BYTES + c * BC * 128, &tm_v, fb, c * 64, hkv, j * BC, b);
-          last_load[slot] = j;
-        } else {
+        for (int t = 0; t < NQT; ++t) {
+          if (j >= wk.nvis_t[t]) continue;
+          if (!mbar_wait(smem_u32(&bars->dec_ready[t]), j & 1, WAIT_TIMEOUT_NS)) {
+            fail = true;
+            break;
+          }
+          const uint32_t keep = *reinterpret_cast<volatile uint32_t*>(&bars->dec_word[t]);
+          mbar_arrive(smem_u32(&bars->dec_ack[t]));
+          if (keep && !loaded) {
+            mbar_arrive_expect_tx(fb, L::V_BYTES);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_4d(v_s + slot * L::V_BYTES + c * BC * 128, &tm_v, fb, c * 64, wk.hkv, j * BC, wk.b);
+            last_load[slot] = j;
+            loaded = true;
+          }
+        }
+        if (fail) {
+          record_failure(p, bars);
+          break;
+        }
+        if (!loaded) {
+          // the MMA warp released this slot's previous load before this use
           mbar_arrive(fb);
+          last_load[slot] = -1;
         }
       }
+      // drain: a load still owning its slot may be in flight only after a
+      // failure; in the normal path this returns at once
       for (int i = 0; i < VST; ++i)
-        if (last_load[i] >= 0)
-          mbar_wait(smem_u32(&bars->v_full[i]), (last_load[i] / VST) & 1, WAIT_TIMEOUT_NS);
-    }
-  } else if (warp == 1) {
-    // ======================= MMA issuer =======================
-    if (lane == 0 && nvis > 0) {
+        if (last_load[i] >= 0 &&
+            !mbar_wait(smem_u32(&bars->v_full[i]), (last_load[i] / VST) & 1, WAIT_TIMEOUT_NS))
+          record_failure(p, bars);
+    } else if (warp == 1 && lane == 0 && nvis > 0) {
+      // ======================= MMA issuer =======================
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BC, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, false, true);
       bool ok = mbar_wait(smem_u32(&bars->q_full), 0, WAIT_TIMEOUT_NS);
-      auto issue_qk = [&](int j) -> bool {
+      int k_ready = -1;  // newest K tile whose arrival was observed
+      auto issue_qk = [&](int t, int j) -> bool {
         const int slot = j % KST;
-        if (!mbar_wait(smem_u32(&bars->k_full[slot]), (j / KST) & 1, WAIT_TIMEOUT_NS)) return false;
+        if (k_ready < j) {
+          if (!mbar_wait(smem_u32(&bars->k_full[slot]), (j / KST) & 1, WAIT_TIMEOUT_NS)) return false;
+          k_ready = j;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + S_COL + 128 * (j & 1);
+        const uint32_t d_tmem = tmem + 256 * t;
+        const uint32_t qt_s = q_s + t * L::QT_BYTES;
 #pragma unroll
         for (int s = 0; s < D / 16; ++s) {
           const uint32_t off = (s >> 2) * (BM * 128) + (s & 3) * 32;
           const uint32_t koff = (s >> 2) * (BC * 128) + (s & 3) * 32;
-          const uint64_t ad = smem_desc_sw128(q_s + off, 16, 1024);
+          const uint64_t ad = smem_desc_sw128(qt_s + off, 16, 1024);
           const uint64_t bd = smem_desc_sw128(k_s + slot * L::K_BYTES + koff, 16, 1024);
           mma_ss(d_tmem, ad, bd, idesc_qk, s > 0 ? 1u : 0u);
         }
-        mma_commit(smem_u32(&bars->k_empty[slot]));
-        mma_commit(smem_u32(&bars->s_full[j & 1]));
+        mma_commit(smem_u32(&bars->s_full[t]));
         return true;
       };
-      if (ok) ok = issue_qk(0);
-      if (ok && nvis > 1) ok = issue_qk(1);
-      int pv_count = 0;
+      // last tile that reads K tile j: B when it visits j, else A
+      auto k_last_user = [&](int j) { return (j < wk.nvis_t[1]) ? 1 : 0; };
+      int pv_count[NQT] = {0, 0};
+#pragma unroll
+      for (int t = 0; t < NQT; ++t)
+        if (ok && wk.nvis_t[t] > 0) {
+          ok = issue_qk(t, 0);
+          if (ok && k_last_user(0) == t) mma_commit(smem_u32(&bars->k_empty[0]));
+        }
       for (int j = 0; ok && j < nvis; ++j) {
         if (aborted(bars)) { ok = false; break; }
-        if (!mbar_wait(smem_u32(&bars->p_ready[j & 1]), (j >> 1) & 1, WAIT_TIMEOUT_NS)) { ok = false; break; }
-        const uint32_t keep = *reinterpret_cast<volatile uint32_t*>(&bars->dec_word[j & 1]);
         const int slot = j % VST;
-        if (!mbar_wait(smem_u32(&bars->v_full[slot]), (j / VST) & 1, WAIT_TIMEOUT_NS)) { ok = false; break; }
-        tc_fence_after();
-        if (keep) {
-          const uint32_t p_tmem = tmem + S_COL + 128 * (j & 1);
+        bool v_seen = false, any_pv = false;
 #pragma unroll
-          for (int s = 0; s < BC / 16; ++s) {
-            const uint64_t bd =
-                smem_desc_sw128(v_s + slot * L::V_BYTES + s * 16 * 128, BC * 128, 1024);
-            mma_ts(tmem + O_COL, p_tmem + s * 8, bd, idesc_pv, (pv_count > 0 || s > 0) ? 1u : 0u);
-          }
-          mma_commit(smem_u32(&bars->v_empty[slot]));
-          mma_commit(smem_u32(&bars->o_bar));
-          ++pv_count;
-        } else {
-          mbar_arrive(smem_u32(&bars->v_empty[slot]));
-        }
-        if (j + 2 < nvis && !issue_qk(j + 2)) { ok = false; break; }
-      }
-      if (!ok) record_failure(p, bars);
-      mma_commit(smem_u32(&bars->o_final));
-      mbar_wait(smem_u32(&bars->o_final), 0, WAIT_TIMEOUT_NS);
-    }
-  } else if (warp >= 4) {
-    // ======================= softmax / epilogue =======================
-    const int row = tid - 128;
-    const int quarter = warp - 4;
-    const int half = p.half ? (row >> 6) : 0;
-    const int grow = pt * BM + row;
-    const bool valid = grow < p.Lq;
-    const int pos = grow + p.Lk - p.Lq;
-    const int pos_first = pt * BM + p.Lk - p.Lq;  // position of the CTA's first row
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16);
-    const bool skip_on = (p.mode & SSA_MODE_SKIP) != 0;
-    const bool nm_on = (p.mode & SSA_MODE_NM) != 0;
-    const bool leader = p.half ? ((row & 63) == 0) : (row == 0);
-    const int my_nvis = nvis_h[half];
-
-    float m_true = -INFINITY;  // running max over kept tiles (raw q.k units)
-    float m_ref = -INFINITY;   // reference the O accumulator and l are scaled to
-    float l = 0.f;
-    int n_pv = 0;
-    int skipped = 0;
-    uint32_t skip_word = 0;
-    bool failed = false;
-
-    for (int j = 0; j < nvis; ++j) {
-      bool ok = !failed && mbar_wait(smem_u32(&bars->s_full[j & 1]), (j >> 1) & 1, WAIT_TIMEOUT_NS);
-      ok = __all_sync(0xffffffffu, ok);
-      float x[BC];
-      float m_tile = -INFINITY;
-      const int col0 = j * BC;
-      if (ok) {
-        tc_fence_after();
-        uint32_t sr[BC];
-#pragma unroll
-        for (int c = 0; c < BC / 32; ++c)
-          tmem_ld32(lane_base + S_COL + 128 * (j & 1) + 32 * c,
-                    *reinterpret_cast<uint32_t(*)[32]>(&sr[32 * c]));
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < BC; ++i) x[i] = __uint_as_float(sr[i]);
-        const bool need_mask = (col0 + BC > p.Lk) || (p.causal && col0 + BC - 1 > pos_first);
-        if (need_mask) {
-#pragma unroll
-          for (int i = 0; i < BC; ++i) {
-            const int jj = col0 + i;
-            if (jj >= p.Lk || (p.causal && jj > pos)) x[i] = -INFINITY;
-          }
-        }
-        if (nm_on) {
-          if (p.m == 4) nm_select<4, BC>(x, p.n, col0, pos, p.sink, p.recent);
-          else nm_select<8, BC>(x, p.n, col0, pos, p.sink, p.recent);
-        }
-#pragma unroll
-        for (int i = 0; i < BC; ++i) m_tile = fmaxf(m_tile, x[i]);
-        if (p.keep_bits != nullptr && valid && j < my_nvis) {
-          uint32_t* kb = p.keep_bits + ((size_t)(b * p.Hq + hq) * p.Lq + grow) * p.Lkw;
-#pragma unroll
-          for (int w = 0; w < BC / 32; ++w) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int t = 0; t < 32; ++t) word |= (x[32 * w + t] != -INFINITY ? 1u : 0u) << t;
-            const int wi = col0 / 32 + w;
-            if (wi < p.Lkw) kb[wi] = word;
-          }
-        }
-      }
-      const bool negligible =
-          !valid || m_tile == -INFINITY ||
-          (m_true != -INFINITY && (m_tile - m_true) * p.scale_log2 < p.log2_lambda);
-      const uint32_t wneg = __all_sync(0xffffffffu, negligible) ? 1u : 0u;
-      if (lane == 0) bars->vote[j & 1][quarter] = wneg | (ok ? 0u : 2u);
-      tc_fence_before();
-      named_bar_sync(1, 128);
-      uint32_t v4[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w) v4[w] = *reinterpret_cast<volatile uint32_t*>(&bars->vote[j & 1][w]);
-      if ((v4[0] | v4[1] | v4[2] | v4[3]) & 2u) {
-        failed = true;
-        if (row == 0) record_failure(p, bars);
-        break;
-      }
-      bool keep_h[2];
-      if (p.half) {
-        keep_h[0] = (j < nvis_h[0]) && !(skip_on && (v4[0] & v4[1] & 1u));
-        keep_h[1] = (j < nvis_h[1]) && !(skip_on && (v4[2] & v4[3] & 1u));
-      } else {
-        keep_h[0] = keep_h[1] = !(skip_on && (v4[0] & v4[1] & v4[2] & v4[3] & 1u));
-      }
-      const bool tile_keep = keep_h[0] || keep_h[1];
-      const bool my_keep = keep_h[half];
-      if (leader && j < my_nvis) {
-        if (!my_keep) {
-          ++skipped;
-          skip_word |= 1u << (j & 31);
-        }
-        if (p.skip_bits != nullptr && ((j & 31) == 31 || j == my_nvis - 1)) {
-          const int qt = p.half ? 2 * pt + half : pt;
-          p.skip_bits[((size_t)(b * p.Hq + hq) * p.nQ + qt) * p.nKw + (j >> 5)] = skip_word;
-          skip_word = 0;
-        }
-      }
-      if (row == 0) {
-        bars->dec_word[j & 1] = tile_keep ? 1u : 0u;
-        mbar_arrive(smem_u32(&bars->dec_ready[j & 1]));
-        if (!tile_keep) mbar_arrive(smem_u32(&bars->p_ready[j & 1]));
-      }
-      if (!tile_keep) continue;
-
-      uint32_t pk[BC / 2];
-      if (my_keep) {
-        const float m_new = fmaxf(m_true, m_tile);
-        m_true = m_new;
-        bool resc = false;
-        if (m_ref == -INFINITY) m_ref = m_true;  // first kept key: O and l are still zero
-        else resc = (m_true - m_ref) * p.scale_log2 > RESCALE_LOG2;
-        if (__any_sync(0xffffffffu, resc)) {
-          bool okw = (n_pv == 0) ||
-                     mbar_wait(smem_u32(&bars->o_bar), (n_pv - 1) & 1, WAIT_TIMEOUT_NS);
-          okw = __all_sync(0xffffffffu, okw);
-          if (!okw) failed = true;  // reported at the next vote
-          const float alpha = resc ? fast_exp2((m_ref - m_true) * p.scale_log2) : 1.f;
-          if (okw && n_pv > 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(lane_base + O_COL + 32 * c, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st32(lane_base + O_COL + 32 * c, o);
+        for (int t = 0; t < NQT; ++t) {
+          if (j >= wk.nvis_t[t]) continue;
+          if (!mbar_wait(smem_u32(&bars->p_ready[t]), j & 1, WAIT_TIMEOUT_NS)) { ok = false; break; }
+          const uint32_t keep = *reinterpret_cast<volatile uint32_t*>(&bars->dec_word[t]);
+          if (keep) {
+            if (!v_seen) {
+              if (!mbar_wait(smem_u32(&bars->v_full[slot]), (j / VST) & 1, WAIT_TIMEOUT_NS)) { ok = false; break; }
+              v_seen = true;
             }
+            tc_fence_after();
+            const uint32_t p_tmem = tmem + 256 * t;
+#pragma unroll
+            for (int s = 0; s < BC / 16; ++s) {
+              const uint64_t bd = smem_desc_sw128(v_s + slot * L::V_BYTES + s * 16 * 128, BC * 128, 1024);
+              mma_ts(tmem + 256 * t + 128, p_tmem + s * 8, bd, idesc_pv,
+                     (pv_count[t] > 0 || s > 0) ? 1u : 0u);
+            }
+            ++pv_count[t];
+            any_pv = true;
           }
-          if (resc) {
-            l *= alpha;
-            m_ref = m_true;
+          if (j == wk.nvis_t[t] - 1) mma_commit(smem_u32(&bars->o_done[t]));
+          if (j + 1 < wk.nvis_t[t]) {
+            if (!issue_qk(t, j + 1)) { ok = false; break; }
+            if (k_last_user(j + 1) == t) mma_commit(smem_u32(&bars->k_empty[(j + 1) % KST]));
           }
         }
-        const float mref_s = (m_ref == -INFINITY) ? 0.f : m_ref * p.scale_log2;
-        float lsum = 0.f;
-#pragma unroll
-        for (int i = 0; i < BC; i += 2) {
-          const float p0 = fast_exp2(fmaf(x[i], p.scale_log2, -mref_s));
-          const float p1 = fast_exp2(fmaf(x[i + 1], p.scale_log2, -mref_s));
-          lsum += p0 + p1;
-          pk[i / 2] = pack_bf16x2(p0, p1);
+        if (!ok) break;
+        if (!v_seen && !mbar_wait(smem_u32(&bars->v_full[slot]), (j / VST) & 1, WAIT_TIMEOUT_NS)) {
+          ok = false;
+          break;
         }
-        l += lsum;
-      } else {
-#pragma unroll
-        for (int i = 0; i < BC / 2; ++i) pk[i] = 0u;
+        if (any_pv) mma_commit(smem_u32(&bars->v_empty[slot]));
+        else mbar_arrive(smem_u32(&bars->v_empty[slot]));
       }
-#pragma unroll
-      for (int c = 0; c < BC / 64; ++c)
-        tmem_st32(lane_base + S_COL + 128 * (j & 1) + 32 * c,
-                  *reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * c]));
-      tmem_wait_st();
-      tc_fence_before();
-      named_bar_sync(2, 128);
-      if (row == 0) mbar_arrive(smem_u32(&bars->p_ready[j & 1]));
-      ++n_pv;
-    }
-
-    // ---- epilogue
-    bool okf = true;
-    if (nvis > 0) okf = mbar_wait(smem_u32(&bars->o_final), 0, WAIT_TIMEOUT_NS);
-    okf = __all_sync(0xffffffffu, okf) && !failed;
-    tc_fence_after();
-    const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = p.out + ((size_t)(b * p.Lq + grow) * p.Hq + hq) * D;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t o[32];
-      if (okf && n_pv > 0) {
-        tmem_ld32(lane_base + O_COL + 32 * c, o);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0u;
-      }
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-        for (int v8 = 0; v8 < 4; ++v8) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(o[8 * v8 + 0]) * inv_l, __uint_as_float(o[8 * v8 + 1]) * inv_l);
-          w.y = pack_bf16x2(__uint_as_float(o[8 * v8 + 2]) * inv_l, __uint_as_float(o[8 * v8 + 3]) * inv_l);
-          w.z = pack_bf16x2(__uint_as_float(o[8 * v8 + 4]) * inv_l, __uint_as_float(o[8 * v8 + 5]) * inv_l);
-          w.w = pack_bf16x2(__uint_as_float(o[8 * v8 + 6]) * inv_l, __uint_as_float(o[8 * v8 + 7]) * inv_l);
-          dst[v8] = w;
-        }
+      if (!ok) {
+        record_failure(p, bars);
+        // unblock the softmax epilogues (they see the failure flag)
+        mma_commit(smem_u32(&bars->o_done[0]));
+        mma_commit(smem_u32(&bars->o_done[1]));
       }
     }
-    if (valid)
-      p.lse[(size_t)(b * p.Hq + hq) * p.Lq + grow] =
-          (l > 0.f) ? m_ref * p.scale + logf(l) : -INFINITY;
-    if (leader) {
-      const int qt = p.half ? 2 * pt + half : pt;
-      if (qt < p.nQ) {
-        p.skip_count[(size_t)(b * p.Hq + hq) * p.nQ + qt] = skipped;
-        if (p.skip_bits != nullptr) {
-          uint32_t* sb = p.skip_bits + ((size_t)(b * p.Hq + hq) * p.nQ + qt) * p.nKw;
-          const int first_unwritten = (my_nvis + 31) / 32;
-          for (int w = first_unwritten; w < p.nKw; ++w) sb[w] = 0u;
-        }
-      }
-    }
+  } else {
+    reg_alloc<200>();
+    const int t = warp >> 3;  // warps 4-7: tile A, 8-11: tile B
+    softmax_tile<D, BC, NM_M, DBG>(p, bars, wk.b, wk.hq, t, t ? wk.pt[1] : wk.pt[0],
+                                   t ? wk.nvis_h[1][0] : wk.nvis_h[0][0],
+                                   t ? wk.nvis_h[1][1] : wk.nvis_h[0][1], tmem);
   }
 
   // ---- teardown
@@ -566,7 +715,7 @@ static std::mutex g_mu;
 static EncodeTiledFn g_encode = nullptr;
 constexpr int MAX_DEV = 64;
 static int* g_status[MAX_DEV] = {};
-static bool g_attr_set[MAX_DEV][4] = {};
+static bool g_attr_set[MAX_DEV][24] = {};
 
 static EncodeTiledFn encode_fn() {
   if (g_encode) return g_encode;
@@ -605,18 +754,36 @@ static int* status_word(int dev) {
   return g_status[dev];
 }
 
-template <int D, int BC>
-static int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                  const Params& p, int grid, cudaStream_t stream, int dev, int inst) {
+template <int D, int BC, int NM_M, bool DBG>
+static int launch_one(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const Params& p, int grid, cudaStream_t stream, int dev, int inst) {
   using L = Smem<D, BC>;
   if (!g_attr_set[dev][inst]) {
-    if (cudaFuncSetAttribute(ssa_fwd_kernel<D, BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)L::ALLOC) != cudaSuccess)
+    if (cudaFuncSetAttribute(ssa_fwd_kernel<D, BC, NM_M, DBG>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC) != cudaSuccess)
       return SSA_ERR_CUDA;
     g_attr_set[dev][inst] = true;
   }
-  ssa_fwd_kernel<D, BC><<<grid, NTHREADS, L::ALLOC, stream>>>(mq, mk, mv, p);
+  ssa_fwd_kernel<D, BC, NM_M, DBG><<<grid, NTHREADS, L::ALLOC, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+// One instance per (N:M group width or none) x (debug outputs or not), so the
+// plain skip-softmax kernel carries no N:M or debug code.
+template <int D, int BC>
+static int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                  const Params& p, int grid, cudaStream_t stream, int dev, int base) {
+  const bool dbg = p.skip_bits != nullptr || p.keep_bits != nullptr;
+  const int nm = (p.mode & SSA_MODE_NM) ? p.m : 0;
+  const int inst = base * 6 + (nm == 0 ? 0 : nm == 4 ? 2 : 4) + (dbg ? 1 : 0);
+  if (nm == 0)
+    return dbg ? launch_one<D, BC, 0, true>(mq, mk, mv, p, grid, stream, dev, inst)
+               : launch_one<D, BC, 0, false>(mq, mk, mv, p, grid, stream, dev, inst);
+  if (nm == 4)
+    return dbg ? launch_one<D, BC, 4, true>(mq, mk, mv, p, grid, stream, dev, inst)
+               : launch_one<D, BC, 4, false>(mq, mk, mv, p, grid, stream, dev, inst);
+  return dbg ? launch_one<D, BC, 8, true>(mq, mk, mv, p, grid, stream, dev, inst)
+             : launch_one<D, BC, 8, false>(mq, mk, mv, p, grid, stream, dev, inst);
 }
 
 static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -642,7 +809,7 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
     if (Bc % m != 0) return SSA_ERR_UNSUPPORTED;
   }
   const long long nQp = (Lq + BM - 1) / BM;
-  const long long grid = nQp * B * Hq;
+  const long long grid = ((nQp + 1) / 2) * B * Hq;
   if (grid > 0x7fffffffLL) return SSA_ERR_UNSUPPORTED;
   if ((long long)B * Lq * Hq * d >= (1LL << 40) || (long long)B * Lk * Hkv * d >= (1LL << 40))
     return SSA_ERR_UNSUPPORTED;
@@ -671,7 +838,6 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
   p.sink = (mode & SSA_MODE_NM) ? sink : 0;
   p.recent = (mode & SSA_MODE_NM) ? recent : 0;
   p.half = (Br == 64) ? 1 : 0;
-  p.Br = Br;
   p.nQp = (int)nQp;
   p.nQ = (Lq + Br - 1) / Br;
   p.nK = (Lk + Bc - 1) / Bc;
