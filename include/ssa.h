@@ -90,6 +90,34 @@ int ssa_fwd_debug(const void* q, const void* k, const void* v, void* out, float*
                   int recent, int Br, int Bc, void* stream, uint32_t* skip_bits,
                   uint32_t* keep_bits);
 
+/* Allocation-free variant of ssa_fwd (the pages have no counterpart; this is
+ * a service of this library).  Same arguments, layouts and results as
+ * ssa_fwd, and it never allocates device memory: no cudaMalloc, no cudaFree,
+ * no allocating library routine.  It is meant for callers that cannot
+ * allocate while they run -- an inference engine's plugin that must work
+ * inside the memory it was given at build time, a process whose device memory
+ * is wholly owned by a framework's pooling allocator, or a latency-critical
+ * path that cannot afford the implicit device synchronisation of cudaMalloc.
+ * ssa_fwd, by contrast, allocates a status word on its first call per device.
+ *
+ * Scratch: the kernel's status word (raised when a bounded device wait times
+ * out) lives in a static 256-byte device array inside libssa, held by every
+ * GPU that loads the library until the process exits.  One call needs 4
+ * bytes of it whatever the problem size; a call needing more than 256 bytes
+ * would be rejected with SSA_ERR_UNSUPPORTED.  The array is shared by every
+ * call on a device and keeps the last call's contents: each call clears the
+ * status word on `stream` before its kernel starts.  Calls that overlap on the
+ * GPU (on different streams) therefore race on that word; serialise them.
+ * A timed-out wait still makes the kernel unwind, but this entry point does
+ * not report it (ssa_device_status reads ssa_fwd's word, not this one).
+ * The first call on a device looks up the array's device address (with that
+ * device current); later calls reuse it.
+ * Returns SSA_OK once enqueued, or the status codes of ssa_fwd. */
+int ssa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                    int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                    int causal, float scale, int mode, float lambda, int n, int m, int sink,
+                    int recent, int Br, int Bc, void* stream);
+
 /* Total key tiles visited by all query tiles of one (batch, head) pair: a pure
  * function of the shape, used to turn skip counts into skip fractions and
  * executed FLOPs.  Returns -1 for invalid sizes. */

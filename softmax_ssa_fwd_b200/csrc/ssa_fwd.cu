@@ -791,7 +791,8 @@ static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr
 static int run(const void* q, const void* k, const void* v, void* out, float* lse,
                int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
                float scale, int mode, float lambda, int n, int m, int sink, int recent, int Br,
-               int Bc, void* stream, uint32_t* skip_bits, uint32_t* keep_bits) {
+               int Bc, void* stream, uint32_t* skip_bits, uint32_t* keep_bits,
+               int* status_override = nullptr) {
   // ---- argument checks (synchronous, nothing launched on failure)
   if (!q || !k || !v || !out || !lse || !tile_skip_count) return SSA_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Lk <= 0 || d <= 0) return SSA_ERR_INVALID_ARG;
@@ -820,7 +821,7 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
   Params p{};
   {
     std::lock_guard<std::mutex> g(g_mu);
-    p.status = status_word(dev);
+    p.status = status_override ? status_override : status_word(dev);
     if (!p.status) return SSA_ERR_CUDA;
     if (!make_map(&mq, q, B, Lq, Hq, d, BM) || !make_map(&mk, k, B, Lk, Hkv, d, Bc) ||
         !make_map(&mv, v, B, Lk, Hkv, d, Bc))
@@ -848,11 +849,59 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
   p.log2_lambda = ((mode & SSA_MODE_SKIP) && lambda > 0.f) ? (float)std::log2((double)lambda)
                                                            : -INFINITY;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // A caller-supplied status word (the allocation-free entry point's shared
+  // scratch) keeps the previous call's contents: clear it on the stream first.
+  if (status_override && cudaMemsetAsync(status_override, 0, sizeof(int), st) != cudaSuccess)
+    return SSA_ERR_CUDA;
   std::lock_guard<std::mutex> g(g_mu);
   if (d == 128 && Bc == 128) return launch<128, 128>(mq, mk, mv, p, (int)grid, st, dev, 0);
   if (d == 128 && Bc == 64) return launch<128, 64>(mq, mk, mv, p, (int)grid, st, dev, 1);
   if (d == 64 && Bc == 128) return launch<64, 128>(mq, mk, mv, p, (int)grid, st, dev, 2);
   return launch<64, 64>(mq, mk, mv, p, (int)grid, st, dev, 3);
+}
+
+
+// ------------------------------------------------------------------------
+// Allocation-free variant.  Its only scratch is the kernel's status word (the
+// flag a CTA raises when one of its bounded waits times out); here it lives in
+// this file-scope device array instead of a lazily cudaMalloc'd word.  Every
+// GPU that loads the library holds the array until the process exits.
+constexpr int NOALLOC_SCRATCH_BYTES = 256;
+static __device__ __align__(256) int g_noalloc_scratch[NOALLOC_SCRATCH_BYTES / sizeof(int)];
+static int* g_noalloc_addr[MAX_DEV] = {};
+
+// Scratch one call needs: the 4-byte status word, whatever the problem size.
+static size_t noalloc_scratch_bytes() { return sizeof(int); }
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device with that device current.
+static int* noalloc_scratch(int dev) {
+  if (dev < 0 || dev >= MAX_DEV) return nullptr;
+  if (!g_noalloc_addr[dev]) {
+    int* ptr = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_noalloc_scratch) != cudaSuccess)
+      return nullptr;
+    g_noalloc_addr[dev] = ptr;
+  }
+  return g_noalloc_addr[dev];
+}
+
+static int run_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                       int causal, float scale, int mode, float lambda, int n, int m, int sink,
+                       int recent, int Br, int Bc, void* stream) {
+  if (noalloc_scratch_bytes() > (size_t)NOALLOC_SCRATCH_BYTES) return SSA_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEV) return SSA_ERR_CUDA;
+  int* scratch;
+  {
+    std::lock_guard<std::mutex> g(g_mu);
+    scratch = noalloc_scratch(dev);
+  }
+  if (!scratch) return SSA_ERR_CUDA;
+  return run(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode, lambda,
+             n, m, sink, recent, Br, Bc, stream, nullptr, nullptr, scratch);
 }
 
 }  // namespace ssa
@@ -874,6 +923,14 @@ int ssa_fwd_debug(const void* q, const void* k, const void* v, void* out, float*
                   uint32_t* keep_bits) {
   return ssa::run(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
                   lambda, n, m, sink, recent, Br, Bc, stream, skip_bits, keep_bits);
+}
+
+int ssa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                    int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                    int causal, float scale, int mode, float lambda, int n, int m, int sink,
+                    int recent, int Br, int Bc, void* stream) {
+  return ssa::run_noalloc(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale,
+                          mode, lambda, n, m, sink, recent, Br, Bc, stream);
 }
 
 int64_t ssa_visited_tiles(int causal, int Lq, int Lk, int Br, int Bc) {

@@ -23,8 +23,8 @@ SSA_ERR_CUDA = -3
 SSA_ERR_TIMEOUT = -4
 MODE_DENSE, MODE_SKIP, MODE_NM = 0, 1, 2
 
-EXPORTED = ["ssa_fwd", "ssa_fwd_debug", "ssa_visited_tiles", "ssa_device_status",
-            "ssa_status_string", "ssa_version"]
+EXPORTED = ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
+            "ssa_device_status", "ssa_status_string", "ssa_version"]
 
 
 class SSAError(RuntimeError):
@@ -43,6 +43,8 @@ def _load():
     lib.ssa_fwd.argtypes = fwd_args
     lib.ssa_fwd_debug.restype = I
     lib.ssa_fwd_debug.argtypes = fwd_args + [P, P]
+    lib.ssa_fwd_noalloc.restype = I
+    lib.ssa_fwd_noalloc.argtypes = fwd_args
     lib.ssa_visited_tiles.restype = ctypes.c_int64
     lib.ssa_visited_tiles.argtypes = [I, I, I, I, I]
     lib.ssa_device_status.restype = I
@@ -95,6 +97,15 @@ def ssa_fwd(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, s
     return lib.ssa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(tile_skip_count),
                        B, Hq, Hkv, Lq, Lk, d, int(causal), float(scale), int(mode), float(lam),
                        int(n), int(m), int(sink), int(recent), Br, Bc, _stream(stream))
+
+
+def ssa_fwd_noalloc(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
+                    lam, n, m, sink, recent, Br, Bc, stream=None) -> int:
+    """The allocation-free entry point (see include/ssa.h); returns its status code."""
+    return lib.ssa_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                               _ptr(tile_skip_count), B, Hq, Hkv, Lq, Lk, d, int(causal),
+                               float(scale), int(mode), float(lam), int(n), int(m), int(sink),
+                               int(recent), Br, Bc, _stream(stream))
 
 
 def ssa_fwd_debug(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
