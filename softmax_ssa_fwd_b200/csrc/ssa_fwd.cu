@@ -125,21 +125,22 @@ __device__ __forceinline__ float mufu_exp2(float x) {
 // f in [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial (max relative error
 // 7.5e-5, below bf16 resolution; coefficients from csrc/fit_exp2_poly.py);
 // 2^n by adding n to the exponent field.  Arguments below -126 give 0.
-__device__ __forceinline__ float2 poly_exp2x2(float x0, float x1) {
+__device__ __forceinline__ float2 poly_exp2x2(uint64_t x01) {
   constexpr float SHIFT = 12582912.0f;  // 1.5 * 2^23
   constexpr float C0 = 0x1.fff692p-1f, C1 = 0x1.62f31ap-1f, C2 = 0x1.f0de1ap-3f, C3 = 0x1.c3f76p-5f;
-  const float a0 = fmaxf(x0, -127.f), a1 = fmaxf(x1, -127.f);
-  float r0, r1, f0, f1, p0, p1;
-  asm("add.rn.f32 %0, %1, %2;" : "=f"(r0) : "f"(a0), "f"(SHIFT));
-  asm("add.rn.f32 %0, %1, %2;" : "=f"(r1) : "f"(a1), "f"(SHIFT));
-  asm("sub.rn.f32 %0, %1, %2;" : "=f"(f0) : "f"(r0), "f"(SHIFT));
-  asm("sub.rn.f32 %0, %1, %2;" : "=f"(f1) : "f"(r1), "f"(SHIFT));
-  f0 = a0 - f0;
-  f1 = a1 - f1;
-  p0 = fmaf(fmaf(fmaf(C3, f0, C2), f0, C1), f0, C0);
-  p1 = fmaf(fmaf(fmaf(C3, f1, C2), f1, C1), f1, C0);
-  const uint32_t b0 = __float_as_uint(p0) + (__float_as_uint(r0) << 23);
-  const uint32_t b1 = __float_as_uint(p1) + (__float_as_uint(r1) << 23);
+  float x0, x1;
+  f2_unpack(x01, x0, x1);
+  const uint64_t a = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const uint64_t r = fadd2(a, f2_pack(SHIFT, SHIFT));            // round to nearest integer
+  const uint64_t f = fsub2(a, fsub2(r, f2_pack(SHIFT, SHIFT)));  // fraction in [-1/2, 1/2]
+  uint64_t q = ffma2(f2_pack(C3, C3), f, f2_pack(C2, C2));
+  q = ffma2(q, f, f2_pack(C1, C1));
+  q = ffma2(q, f, f2_pack(C0, C0));
+  float q0, q1, r0, r1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(r, r0, r1);
+  const uint32_t b0 = __float_as_uint(q0) + (__float_as_uint(r0) << 23);
+  const uint32_t b1 = __float_as_uint(q1) + (__float_as_uint(r1) << 23);
   return make_float2(x0 < -126.f ? 0.f : __uint_as_float(b0), x1 < -126.f ? 0.f : __uint_as_float(b1));
 }
 
@@ -165,32 +166,80 @@ __device__ __forceinline__ void reg_alloc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// N:M selection on one thread's row: for each aligned group of M keys keep a
-// key iff (inside the sink / recent window, or among the N largest scores of
-// its group, equal scores ranked by lower index); dropped keys become -inf.
-// Masked keys are already -inf, rank last and stay -inf.
-template <int M, int BC>
-__device__ __forceinline__ void nm_select(float (&x)[BC], int N, int col0, int pos, int sink,
-                                          int recent) {
+// Sorting networks (descending) used to find the N-th largest score of an
+// N:M group: 5 comparators for 4 inputs, Batcher's odd-even merge sort (19
+// comparators) for 8.
+__device__ __forceinline__ void cmpx(float& hi, float& lo) {
+  const float h = fmaxf(hi, lo), l = fminf(hi, lo);
+  hi = h;
+  lo = l;
+}
+template <int M>
+__device__ __forceinline__ void sort_desc(float (&s)[M]) {
+  if constexpr (M == 4) {
+    cmpx(s[0], s[1]); cmpx(s[2], s[3]); cmpx(s[0], s[2]); cmpx(s[1], s[3]); cmpx(s[1], s[2]);
+  } else {
+    cmpx(s[0], s[1]); cmpx(s[2], s[3]); cmpx(s[4], s[5]); cmpx(s[6], s[7]);
+    cmpx(s[0], s[2]); cmpx(s[1], s[3]); cmpx(s[1], s[2]);
+    cmpx(s[4], s[6]); cmpx(s[5], s[7]); cmpx(s[5], s[6]);
+    cmpx(s[0], s[4]); cmpx(s[1], s[5]); cmpx(s[2], s[6]); cmpx(s[3], s[7]);
+    cmpx(s[2], s[4]); cmpx(s[3], s[5]);
+    cmpx(s[1], s[2]); cmpx(s[3], s[4]); cmpx(s[5], s[6]);
+  }
+}
+
+// N:M selection on one thread's row (64 columns): for each aligned group of
+// M keys keep a key iff it is inside the sink / recent window or among the N
+// largest scores of its group, equal scores ranked by lower index; dropped
+// keys become -inf.  Masked keys are already -inf and stay -inf.
+// Fast path: with thr the N-th largest and nxt the (N+1)-th, thr > nxt means
+// the top N are exactly the keys >= thr (thr = -inf: every finite key).  A
+// tie (thr == nxt, finite) falls back to explicit ranks.
+template <int M>
+__device__ __forceinline__ void nm_select(float (&x)[64], int N, int col0, int pos, int sink,
+                                          int recent, bool windows) {
 #pragma unroll
-  for (int g = 0; g < BC / M; ++g) {
-    int rank[M];
+  for (int g = 0; g < 64 / M; ++g) {
+    float srt[M];
 #pragma unroll
-    for (int a = 0; a < M; ++a) rank[a] = 0;
+    for (int a = 0; a < M; ++a) srt[a] = x[g * M + a];
+    sort_desc<M>(srt);
+    float thr = srt[0], nxt = srt[1];
+#pragma unroll
+    for (int r = 1; r < M; ++r)
+      if (N == r + 1) {
+        thr = srt[r];
+        nxt = r + 1 < M ? srt[r + 1] : -INFINITY;
+      }
+    bool keep[M];
+    if (thr == nxt && thr != -INFINITY) {
+      int rank[M];
+#pragma unroll
+      for (int a = 0; a < M; ++a) rank[a] = 0;
+#pragma unroll
+      for (int a = 0; a < M; ++a)
+#pragma unroll
+        for (int c = a + 1; c < M; ++c) {
+          if (x[g * M + c] > x[g * M + a]) ++rank[a];
+          else ++rank[c];
+        }
+#pragma unroll
+      for (int a = 0; a < M; ++a) keep[a] = rank[a] < N;
+    } else {
+#pragma unroll
+      for (int a = 0; a < M; ++a) keep[a] = x[g * M + a] >= thr;
+    }
+    if (windows) {
+#pragma unroll
+      for (int a = 0; a < M; ++a) {
+        const int jj = col0 + g * M + a;
+        const int dist = pos - jj;
+        keep[a] = keep[a] || (jj < sink) || (dist >= 0 && dist < recent);
+      }
+    }
 #pragma unroll
     for (int a = 0; a < M; ++a)
-#pragma unroll
-      for (int c = a + 1; c < M; ++c) {
-        if (x[g * M + c] > x[g * M + a]) ++rank[a];
-        else ++rank[c];
-      }
-#pragma unroll
-    for (int a = 0; a < M; ++a) {
-      const int jj = col0 + g * M + a;
-      const int dist = pos - jj;
-      const bool win = (jj < sink) || (dist >= 0 && dist < recent);
-      if (!(win || rank[a] < N)) x[g * M + a] = -INFINITY;
-    }
+      if (!keep[a]) x[g * M + a] = -INFINITY;
   }
 }
 
@@ -221,7 +270,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
   const bool leader = p.half ? ((row & 63) == 0) : (row == 0);
   const int my_nvis = half ? nvis_h1 : nvis_h0;
   const int nvis = nvis_h0 > nvis_h1 ? nvis_h0 : nvis_h1;
-  const uint32_t bar_vote = 1 + t, bar_p = 3 + t;
+  const uint32_t bar_vote = 1 + t;
 
   float m_true = -INFINITY;  // running max over kept tiles (raw q.k units)
   float m_ref = -INFINITY;   // reference the O accumulator and l are scaled to
@@ -239,9 +288,12 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     // Pass 1, 64 columns at a time: masks, N:M, tile row max.  Masked
     // scores are written back to TMEM so pass 2 needs no mask.
     const bool need_mask = (col0 + BC > p.Lk) || (p.causal && col0 + BC - 1 > pos_first);
+    // does this key tile meet the sink or any row's recent window?
+    const bool nm_windows = nm_on && ((col0 < p.sink) ||
+                                      (col0 <= pos_first + BM - 1 && col0 + BC - 1 > pos_first - p.recent));
     if (ok) {
       tc_fence_after();
-#pragma unroll
+#pragma unroll 1
       for (int bb = 0; bb < BC / 64; ++bb) {
         float x[64];
         const uint32_t ta = lane_base + s_col + 64 * bb;
@@ -256,14 +308,15 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
             if (jj >= p.Lk || (p.causal && jj > pos)) x[i] = -INFINITY;
           }
         }
-        if constexpr (nm_on) nm_select<(NM_M ? NM_M : 4), 64>(x, p.n, cb, pos, p.sink, p.recent);
+        if constexpr (nm_on)
+          nm_select<(NM_M ? NM_M : 4)>(x, p.n, cb, pos, p.sink, p.recent, nm_windows);
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
         for (int i = 0; i < 64; i += 4) {
-          mx0 = fmaxf(mx0, fmaxf(x[i], x[i + 1]));
-          mx1 = fmaxf(mx1, fmaxf(x[i + 2], x[i + 3]));
+          mx0 = fmax3(mx0, x[i], x[i + 1]);
+          mx1 = fmax3(mx1, x[i + 2], x[i + 3]);
         }
-        m_tile = fmaxf(m_tile, fmaxf(mx0, mx1));
+        m_tile = fmax3(m_tile, mx0, mx1);
         if (need_mask || nm_on) {
           tmem_st32(ta, *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
           tmem_st32(ta + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));
@@ -324,9 +377,11 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
         record_failure(p, bars);
       bars->dec_word[t] = tile_keep ? 1u : 0u;
       mbar_arrive(smem_u32(&bars->dec_ready[t]));
-      if (!tile_keep) mbar_arrive(smem_u32(&bars->p_ready[t]));
     }
-    if (!tile_keep) continue;
+    if (!tile_keep) {
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[t]));
+      continue;
+    }
 
     if (my_keep) {
       m_true = fmaxf(m_true, m_tile);
@@ -355,8 +410,9 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       // Pass 2: P = exp2((s - m_ref) * scale * log2 e), 64 columns at a time
       const float c = p.scale_log2;
       const float mref_s = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-      float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
+      const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-mref_s, -mref_s);
+      uint64_t ls2 = f2_pack(0.f, 0.f);
+#pragma unroll 1
       for (int bb = 0; bb < BC / 64; ++bb) {
         float x[64];
         const uint32_t ta = lane_base + s_col + 64 * bb;
@@ -366,23 +422,25 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float a0 = fmaf(x[2 * i], c, -mref_s);
-          const float a1 = fmaf(x[2 * i + 1], c, -mref_s);
+          const uint64_t a2 = ffma2(f2_pack(x[2 * i], x[2 * i + 1]), c2, nm2);
           float p0, p1;
           if ((i % POLY_EVERY) == POLY_EVERY - 1) {
-            const float2 ev = poly_exp2x2(a0, a1);
+            const float2 ev = poly_exp2x2(a2);
             p0 = ev.x;
             p1 = ev.y;
           } else {
+            float a0, a1;
+            f2_unpack(a2, a0, a1);
             p0 = mufu_exp2(a0);
             p1 = mufu_exp2(a1);
           }
-          ls0 += p0;
-          ls1 += p1;
+          ls2 = fadd2(ls2, f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st32(lane_base + s_col + 32 * bb, pk);
       }
+      float ls0, ls1;
+      f2_unpack(ls2, ls0, ls1);
       l += ls0 + ls1;
     } else {
       uint32_t pk[32];
@@ -393,8 +451,8 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     }
     tmem_wait_st();
     tc_fence_before();
-    named_bar_sync(bar_p, 128);
-    if (row == 0) mbar_arrive(smem_u32(&bars->p_ready[t]));
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[t]));
     ++n_pv;
   }
 
@@ -504,7 +562,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(smem_u32(&bars->s_full[i]), 1);
       mbar_init(smem_u32(&bars->dec_ready[i]), 1);
       mbar_init(smem_u32(&bars->dec_ack[i]), 1);
-      mbar_init(smem_u32(&bars->p_ready[i]), 1);
+      mbar_init(smem_u32(&bars->p_ready[i]), 4);  // one arrival per softmax warp
       mbar_init(smem_u32(&bars->o_done[i]), 1);
     }
     bars->abort_flag = 0;
