@@ -291,7 +291,26 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     // does this key tile meet the sink or any row's recent window?
     const bool nm_windows = nm_on && ((col0 < p.sink) ||
                                       (col0 <= pos_first + BM - 1 && col0 + BC - 1 > pos_first - p.recent));
-    if (ok) {
+    if (ok && !nm_on && !need_mask) {
+      // common case: one TMEM round trip for the whole row, max only
+      tc_fence_after();
+      float xa[BC];
+#pragma unroll
+      for (int c = 0; c < BC / 32; ++c) tmem_ld32f(lane_base + s_col + 32 * c, &xa[32 * c]);
+      tmem_wait_ld();
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < BC; i += 4) {
+        mx0 = fmax3(mx0, xa[i], xa[i + 1]);
+        mx1 = fmax3(mx1, xa[i + 2], xa[i + 3]);
+      }
+      m_tile = fmax3(m_tile, mx0, mx1);
+      if (DBG && p.keep_bits != nullptr && valid && j < my_nvis) {
+        uint32_t* kb = p.keep_bits + ((size_t)(b * p.Hq + hq) * p.Lq + grow) * p.Lkw;
+#pragma unroll
+        for (int w = 0; w < BC / 32; ++w) kb[col0 / 32 + w] = 0xffffffffu;
+      }
+    } else if (ok) {
       tc_fence_after();
 #pragma unroll 1
       for (int bb = 0; bb < BC / 64; ++bb) {
@@ -379,6 +398,8 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       mbar_arrive(smem_u32(&bars->dec_ready[t]));
     }
     if (!tile_keep) {
+      tc_fence_before();
+      __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[t]));
       continue;
     }
@@ -388,24 +409,14 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       bool resc = false;
       if (m_ref == -INFINITY) m_ref = m_true;  // first kept key: O and l are still zero
       else resc = (m_true - m_ref) * p.scale_log2 > RESCALE_LOG2;
-      if (__any_sync(0xffffffffu, resc)) {
-        // every earlier P.V of this tile completed before S(j) did
-        const float alpha = resc ? mufu_exp2((m_ref - m_true) * p.scale_log2) : 1.f;
-        if (n_pv > 0) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + o_col + 32 * c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(lane_base + o_col + 32 * c, o);
-          }
-        }
-        if (resc) {
-          l *= alpha;
-          m_ref = m_true;
-        }
+      // O is rescaled after P is written (the S registers are free then);
+      // every earlier P.V of this tile completed before S(j) did.
+      const bool any_resc = __any_sync(0xffffffffu, resc);
+      float alpha = 1.f;
+      if (resc) {
+        alpha = mufu_exp2((m_ref - m_true) * p.scale_log2);
+        l *= alpha;
+        m_ref = m_true;
       }
       // Pass 2: P = exp2((s - m_ref) * scale * log2 e), 64 columns at a time
       const float c = p.scale_log2;
@@ -415,10 +426,12 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
 #pragma unroll 1
       for (int bb = 0; bb < BC / 64; ++bb) {
         float x[64];
-        const uint32_t ta = lane_base + s_col + 64 * bb;
-        tmem_ld32f(ta, &x[0]);
-        tmem_ld32f(ta + 32, &x[32]);
-        tmem_wait_ld();
+        {
+          const uint32_t ta = lane_base + s_col + 64 * bb;
+          tmem_ld32f(ta, &x[0]);
+          tmem_ld32f(ta + 32, &x[32]);
+          tmem_wait_ld();
+        }
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -442,6 +455,17 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       float ls0, ls1;
       f2_unpack(ls2, ls0, ls1);
       l += ls0 + ls1;
+      if (any_resc && n_pv > 0) {
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + o_col + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(lane_base + o_col + 32 * c, o);
+        }
+      }
     } else {
       uint32_t pk[32];
 #pragma unroll
