@@ -57,6 +57,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait with an explicit bound on how long the hardware may suspend the
+// thread before re-checking (nanoseconds); short bounds keep wake-up latency low.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for latency-critical single-thread roles.
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  if (mbar_try_wait_hint(bar, parity, 20)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait_hint(bar, parity, 20)) return true;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+}
+
 // Waits for the phase of the given parity to complete, for at most
 // timeout_ns.  Returns false on timeout; the caller records the error and
 // unwinds instead of hanging.

@@ -55,8 +55,11 @@ constexpr int NTHREADS = 384;
 constexpr int TMEM_COLS = 512;
 constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;  // 2 s per wait
 constexpr float RESCALE_LOG2 = 8.0f;  // lazy O rescale once the max grew by 2^8
-// One exp2 in POLY_EVERY pairs runs as a polynomial on the FMA pipe.
-constexpr int POLY_EVERY = 4;
+// When POLY_EVERY > 0, one exp2 pair in POLY_EVERY runs as a polynomial on
+// the FMA pipe instead of the MUFU unit.  Measured on B200 (llama8k, wan) the
+// softmax here is latency-bound, not MUFU-bound, and every offload ratio
+// tried (1/2, 1/3, 1/4, 1/8) was slower than none, so it is off.
+constexpr int POLY_EVERY = 0;
 
 struct Params {
   __nv_bfloat16* out;
@@ -392,7 +395,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     if (row == 0) {
       // the V producer must have taken decision j-1 before decision j is
       // published on the same barrier (keeps its phases from aliasing)
-      if (j > 0 && !mbar_wait(smem_u32(&bars->dec_ack[t]), (j - 1) & 1, WAIT_TIMEOUT_NS))
+      if (j > 0 && !mbar_wait_fast(smem_u32(&bars->dec_ack[t]), (j - 1) & 1, WAIT_TIMEOUT_NS))
         record_failure(p, bars);
       bars->dec_word[t] = tile_keep ? 1u : 0u;
       mbar_arrive(smem_u32(&bars->dec_ready[t]));
@@ -423,21 +426,19 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       const float mref_s = (m_ref == -INFINITY) ? 0.f : m_ref * c;
       const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-mref_s, -mref_s);
       uint64_t ls2 = f2_pack(0.f, 0.f);
-#pragma unroll 1
+      // all of S in one TMEM round trip, then 32 bf16 pairs per 64 columns
+      float x[BC];
+#pragma unroll
+      for (int cc = 0; cc < BC / 32; ++cc) tmem_ld32f(lane_base + s_col + 32 * cc, &x[32 * cc]);
+      tmem_wait_ld();
+#pragma unroll
       for (int bb = 0; bb < BC / 64; ++bb) {
-        float x[64];
-        {
-          const uint32_t ta = lane_base + s_col + 64 * bb;
-          tmem_ld32f(ta, &x[0]);
-          tmem_ld32f(ta + 32, &x[32]);
-          tmem_wait_ld();
-        }
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const uint64_t a2 = ffma2(f2_pack(x[2 * i], x[2 * i + 1]), c2, nm2);
+          const uint64_t a2 = ffma2(f2_pack(x[64 * bb + 2 * i], x[64 * bb + 2 * i + 1]), c2, nm2);
           float p0, p1;
-          if ((i % POLY_EVERY) == POLY_EVERY - 1) {
+          if (POLY_EVERY > 0 && (i % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1) {
             const float2 ev = poly_exp2x2(a2);
             p0 = ev.x;
             p1 = ev.y;
@@ -657,7 +658,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
           if (j >= wk.nvis_t[t]) continue;
-          if (!mbar_wait(smem_u32(&bars->dec_ready[t]), j & 1, WAIT_TIMEOUT_NS)) {
+          if (!mbar_wait_fast(smem_u32(&bars->dec_ready[t]), j & 1, WAIT_TIMEOUT_NS)) {
             fail = true;
             break;
           }
@@ -697,7 +698,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       auto issue_qk = [&](int t, int j) -> bool {
         const int slot = j % KST;
         if (k_ready < j) {
-          if (!mbar_wait(smem_u32(&bars->k_full[slot]), (j / KST) & 1, WAIT_TIMEOUT_NS)) return false;
+          if (!mbar_wait_fast(smem_u32(&bars->k_full[slot]), (j / KST) & 1, WAIT_TIMEOUT_NS)) return false;
           k_ready = j;
         }
         tc_fence_after();
@@ -730,11 +731,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
           if (j >= wk.nvis_t[t]) continue;
-          if (!mbar_wait(smem_u32(&bars->p_ready[t]), j & 1, WAIT_TIMEOUT_NS)) { ok = false; break; }
+          if (!mbar_wait_fast(smem_u32(&bars->p_ready[t]), j & 1, WAIT_TIMEOUT_NS)) { ok = false; break; }
           const uint32_t keep = *reinterpret_cast<volatile uint32_t*>(&bars->dec_word[t]);
           if (keep) {
             if (!v_seen) {
-              if (!mbar_wait(smem_u32(&bars->v_full[slot]), (j / VST) & 1, WAIT_TIMEOUT_NS)) { ok = false; break; }
+              if (!mbar_wait_fast(smem_u32(&bars->v_full[slot]), (j / VST) & 1, WAIT_TIMEOUT_NS)) { ok = false; break; }
               v_seen = true;
             }
             tc_fence_after();
@@ -755,7 +756,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         if (!ok) break;
-        if (!v_seen && !mbar_wait(smem_u32(&bars->v_full[slot]), (j / VST) & 1, WAIT_TIMEOUT_NS)) {
+        if (!v_seen && !mbar_wait_fast(smem_u32(&bars->v_full[slot]), (j / VST) & 1, WAIT_TIMEOUT_NS)) {
           ok = false;
           break;
         }
