@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 from softmax_ssa_fwd_b200.inputs import MODE_NM, MODE_SKIP, WORKLOADS, make_inputs  # noqa: E402
 
 KERNEL_SRC = [os.path.join(ROOT, "softmax_ssa_fwd_b200", "csrc", f) for f in ("ssa_fwd.cu", "ptx.cuh")]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ssa_fwd_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ssa_fwd_traffic.json")  # ncu DRAM bytes, keyed by kernel source hash
 
 
 def kernel_hash() -> str:
@@ -66,6 +66,20 @@ def dense_equiv_flops(w, Lq=None) -> float:
     else:
         pairs = Lq * Lk
     return 4.0 * w.d * w.B * w.Hq * pairs
+
+
+def reduce_max(x: float, dist, device) -> float:
+    """Max over ranks (the job's time is its slowest rank's); identity without a group."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank processes its own replica of the workload."""
+    return world * units_per_rank / (ms_max * 1e-3)
 
 
 def workload_name(w, lam):
@@ -281,10 +295,7 @@ def main():
     ms = e0.elapsed_time(e1)
     if ssa.ssa_device_status(stream) != 0:
         raise RuntimeError("device-side timeout in the timed region")
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(ms, dist, dev)
     ms_step = ms / args.steps
 
     # skip statistics of the timed workload (identical every step per input set)
@@ -293,10 +304,10 @@ def main():
     kept = visited - skipped
     flops_dense = dense_equiv_flops(w)
     flops_exec = 2.0 * w.Br * w.Bc * w.d * (visited + kept)
-    tflops_dense = world * flops_dense / (ms_step * 1e-3) / 1e12
-    tflops_exec = world * flops_exec / (ms_step * 1e-3) / 1e12
+    tflops_dense = job_rate(flops_dense, world, ms_step) / 1e12
+    tflops_exec = job_rate(flops_exec, world, ms_step) / 1e12
     bf16_peak, bf16_sus, hbm_peak, src = peaks()
-    tokens = world * w.B * w.L / (ms_step * 1e-3)
+    tokens = job_rate(w.B * w.L, world, ms_step)
 
     traffic = None
     if os.path.exists(TRAFFIC_FILE):
@@ -339,12 +350,8 @@ def main():
         e1.record(stream)
         e1.synchronize()
         barrier()
-        ems = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * flops_dense / (ems / n_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+        ems = reduce_max(e0.elapsed_time(e1), dist, dev)
+        e2e = {"value": job_rate(flops_dense, world, ems / n_e2e) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems / n_e2e,
                "steps": n_e2e}
 
@@ -370,7 +377,7 @@ def main():
                          "peak": bf16_peak, "unit": "TFLOP/s",
                          "frac": flops_exec / (ms_step * 1e-3) / 1e12 / bf16_peak,
                          "traffic": traffic, "peak_source": f"{src} bf16 burst",
-                         "kernel": "ssa::ssa_fwd_kernel<128,128>",
+                         "kernel": "ssa::ssa_fwd_kernel<128,128,0,0>",
                          "dense_equiv_frac": flops_dense / (ms_step * 1e-3) / 1e12 / bf16_peak,
                          "hbm_frac_of_algorithmic_bytes": None},
             "gpu_launches": args.steps,
