@@ -123,6 +123,16 @@ int ssa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, floa
  * executed FLOPs.  Returns -1 for invalid sizes. */
 int64_t ssa_visited_tiles(int causal, int Lq, int Lk, int Br, int Bc);
 
+/* Test and diagnosis knob: the limit, in nanoseconds, of each pipeline wait
+ * inside the kernel (an mbarrier wait for a TMA load, an MMA result, a
+ * softmax hand-off).  0 restores the default (2 s).  When a wait gives up the
+ * CTA unwinds: it records SSA_ERR_TIMEOUT, waits (with a separate, fixed 2 s
+ * limit) for its own TMA loads and MMAs to finish, frees its tensor memory
+ * and exits, so the context stays usable.  A tiny limit forces that path
+ * without any fault; its outputs are then undefined.  Process-wide; takes
+ * effect at the next launch. */
+void ssa_set_wait_timeout_ns(uint64_t ns);
+
 /* Synchronises `stream`, returns SSA_OK or SSA_ERR_TIMEOUT if a kernel on this
  * device recorded a timed-out wait since the last call, and clears the word.
  * Returns SSA_ERR_CUDA if the synchronisation itself fails. */

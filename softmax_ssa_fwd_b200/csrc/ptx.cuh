@@ -75,9 +75,7 @@ __device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity, ui
   if (mbar_try_wait_hint(bar, parity, 20)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait_hint(bar, parity, 20)) return true;
+    if (mbar_try_wait_hint(bar, parity, 20)) return true;
     if (globaltimer_ns() - t0 > timeout_ns) return false;
   }
 }
@@ -89,9 +87,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (globaltimer_ns() - t0 > timeout_ns) return false;
   }
 }

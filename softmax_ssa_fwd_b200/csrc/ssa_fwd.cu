@@ -53,7 +53,10 @@ constexpr int KST = 2;        // K ring depth
 constexpr int VST = 2;        // V ring depth
 constexpr int NTHREADS = 384;
 constexpr int TMEM_COLS = 512;
-constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;  // 2 s per wait
+constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;  // default limit of a pipeline wait (2 s)
+// Limit of the waits that make a failing CTA's own asynchronous work (TMA
+// loads, MMAs) finish before it frees its memory; never shortened.
+constexpr uint64_t DRAIN_TIMEOUT_NS = 2000000000ull;
 constexpr float RESCALE_LOG2 = 8.0f;  // lazy O rescale once the max grew by 2^8
 // When POLY_EVERY > 0, one exp2 pair in POLY_EVERY runs as a polynomial on
 // the FMA pipe instead of the MUFU unit.  Measured on B200 (llama8k, wan) the
@@ -78,6 +81,7 @@ struct Params {
   float scale;
   float scale_log2;
   float log2_lambda;  // -inf for lambda == 0
+  unsigned long long wait_ns;  // limit of each pipeline wait
 };
 
 struct __align__(8) Bars {
@@ -85,6 +89,7 @@ struct __align__(8) Bars {
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
   uint64_t s_full[NQT], dec_ready[NQT], dec_ack[NQT], p_ready[NQT], o_done[NQT];
+  uint64_t mma_done;
   uint32_t tmem_base;
   uint32_t dec_word[NQT];
   uint32_t vote[NQT][2][4];
@@ -284,7 +289,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
   bool failed = false;
 
   for (int j = 0; j < nvis; ++j) {
-    bool ok = !failed && mbar_wait(smem_u32(&bars->s_full[t]), j & 1, WAIT_TIMEOUT_NS);
+    bool ok = !failed && mbar_wait(smem_u32(&bars->s_full[t]), j & 1, p.wait_ns);
     ok = __all_sync(0xffffffffu, ok);
     float m_tile = -INFINITY;
     const int col0 = j * BC;
@@ -395,7 +400,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     if (row == 0) {
       // the V producer must have taken decision j-1 before decision j is
       // published on the same barrier (keeps its phases from aliasing)
-      if (j > 0 && !mbar_wait_fast(smem_u32(&bars->dec_ack[t]), (j - 1) & 1, WAIT_TIMEOUT_NS))
+      if (j > 0 && !mbar_wait_fast(smem_u32(&bars->dec_ack[t]), (j - 1) & 1, p.wait_ns))
         record_failure(p, bars);
       bars->dec_word[t] = tile_keep ? 1u : 0u;
       mbar_arrive(smem_u32(&bars->dec_ready[t]));
@@ -483,7 +488,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
 
   // ---- epilogue
   bool okf = true;
-  if (nvis > 0) okf = mbar_wait(smem_u32(&bars->o_done[t]), 0, WAIT_TIMEOUT_NS);
+  if (nvis > 0) okf = mbar_wait(smem_u32(&bars->o_done[t]), 0, p.wait_ns);
   if (!okf) record_failure(p, bars);
   okf = __all_sync(0xffffffffu, okf) && !failed;
   tc_fence_after();
@@ -590,6 +595,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(smem_u32(&bars->p_ready[i]), 4);  // one arrival per softmax warp
       mbar_init(smem_u32(&bars->o_done[i]), 1);
     }
+    mbar_init(smem_u32(&bars->mma_done), 1);
     bars->abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -626,7 +632,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int j = 0; j < nvis; ++j) {
         const int slot = j % KST;
         if (aborted(bars)) break;
-        if (!mbar_wait(smem_u32(&bars->k_empty[slot]), ((j / KST) & 1) ^ 1, WAIT_TIMEOUT_NS)) {
+        if (!mbar_wait(smem_u32(&bars->k_empty[slot]), ((j / KST) & 1) ^ 1, p.wait_ns)) {
           record_failure(p, bars);
           break;
         }
@@ -638,9 +644,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         issued = j + 1;
       }
       // drain: the newest load of each slot (older ones were consumed)
-      bool drained = mbar_wait(qbar, 0, WAIT_TIMEOUT_NS);
+      bool drained = mbar_wait(qbar, 0, DRAIN_TIMEOUT_NS);
       for (int j = issued - KST; j < issued; ++j)
-        if (j >= 0) drained &= mbar_wait(smem_u32(&bars->k_full[j % KST]), (j / KST) & 1, WAIT_TIMEOUT_NS);
+        if (j >= 0) drained &= mbar_wait(smem_u32(&bars->k_full[j % KST]), (j / KST) & 1, DRAIN_TIMEOUT_NS);
       if (!drained) record_failure(p, bars);
     } else if (warp == 2 && lane == 0) {
       // ======================= V producer =======================
@@ -649,7 +655,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       for (int j = 0; j < nvis; ++j) {
         if (aborted(bars)) break;
         const int slot = j % VST;
-        if (!mbar_wait(smem_u32(&bars->v_empty[slot]), ((j / VST) & 1) ^ 1, WAIT_TIMEOUT_NS)) {
+        if (!mbar_wait(smem_u32(&bars->v_empty[slot]), ((j / VST) & 1) ^ 1, p.wait_ns)) {
           record_failure(p, bars);
           break;
         }
@@ -658,7 +664,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
           if (j >= wk.nvis_t[t]) continue;
-          if (!mbar_wait_fast(smem_u32(&bars->dec_ready[t]), j & 1, WAIT_TIMEOUT_NS)) {
+          if (!mbar_wait_fast(smem_u32(&bars->dec_ready[t]), j & 1, p.wait_ns)) {
             fail = true;
             break;
           }
@@ -687,18 +693,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // failure; in the normal path this returns at once
       for (int i = 0; i < VST; ++i)
         if (last_load[i] >= 0 &&
-            !mbar_wait(smem_u32(&bars->v_full[i]), (last_load[i] / VST) & 1, WAIT_TIMEOUT_NS))
+            !mbar_wait(smem_u32(&bars->v_full[i]), (last_load[i] / VST) & 1, DRAIN_TIMEOUT_NS))
           record_failure(p, bars);
     } else if (warp == 1 && lane == 0 && nvis > 0) {
       // ======================= MMA issuer =======================
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BC, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, false, true);
-      bool ok = mbar_wait(smem_u32(&bars->q_full), 0, WAIT_TIMEOUT_NS);
+      bool ok = mbar_wait(smem_u32(&bars->q_full), 0, p.wait_ns);
       int k_ready = -1;  // newest K tile whose arrival was observed
       auto issue_qk = [&](int t, int j) -> bool {
         const int slot = j % KST;
         if (k_ready < j) {
-          if (!mbar_wait_fast(smem_u32(&bars->k_full[slot]), (j / KST) & 1, WAIT_TIMEOUT_NS)) return false;
+          if (!mbar_wait_fast(smem_u32(&bars->k_full[slot]), (j / KST) & 1, p.wait_ns)) return false;
           k_ready = j;
         }
         tc_fence_after();
@@ -731,11 +737,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
           if (j >= wk.nvis_t[t]) continue;
-          if (!mbar_wait_fast(smem_u32(&bars->p_ready[t]), j & 1, WAIT_TIMEOUT_NS)) { ok = false; break; }
+          if (!mbar_wait_fast(smem_u32(&bars->p_ready[t]), j & 1, p.wait_ns)) { ok = false; break; }
           const uint32_t keep = *reinterpret_cast<volatile uint32_t*>(&bars->dec_word[t]);
           if (keep) {
             if (!v_seen) {
-              if (!mbar_wait_fast(smem_u32(&bars->v_full[slot]), (j / VST) & 1, WAIT_TIMEOUT_NS)) { ok = false; break; }
+              if (!mbar_wait_fast(smem_u32(&bars->v_full[slot]), (j / VST) & 1, p.wait_ns)) { ok = false; break; }
               v_seen = true;
             }
             tc_fence_after();
@@ -756,7 +762,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
         }
         if (!ok) break;
-        if (!v_seen && !mbar_wait_fast(smem_u32(&bars->v_full[slot]), (j / VST) & 1, WAIT_TIMEOUT_NS)) {
+        if (!v_seen && !mbar_wait_fast(smem_u32(&bars->v_full[slot]), (j / VST) & 1, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -769,6 +775,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mma_commit(smem_u32(&bars->o_done[0]));
         mma_commit(smem_u32(&bars->o_done[1]));
       }
+      // every MMA this thread issued has completed before TMEM is freed
+      mma_commit(smem_u32(&bars->mma_done));
+      if (!mbar_wait(smem_u32(&bars->mma_done), 0, DRAIN_TIMEOUT_NS)) record_failure(p, bars);
     }
   } else {
     reg_alloc<200>();
@@ -795,6 +804,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static std::mutex g_mu;
+static unsigned long long g_wait_ns = WAIT_TIMEOUT_NS;
 static EncodeTiledFn g_encode = nullptr;
 constexpr int MAX_DEV = 64;
 static int* g_status[MAX_DEV] = {};
@@ -931,6 +941,7 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
   p.scale_log2 = (float)((double)scale * 1.4426950408889634);
   p.log2_lambda = ((mode & SSA_MODE_SKIP) && lambda > 0.f) ? (float)std::log2((double)lambda)
                                                            : -INFINITY;
+  p.wait_ns = g_wait_ns;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // A caller-supplied status word (the allocation-free entry point's shared
   // scratch) keeps the previous call's contents: clear it on the stream first.
@@ -1022,6 +1033,11 @@ int64_t ssa_visited_tiles(int causal, int Lq, int Lk, int Br, int Bc) {
   int64_t t = 0;
   for (int qt = 0; qt < nQ; ++qt) t += ssa::visited_key_tiles(causal, Lq, Lk, Br, Bc, qt);
   return t;
+}
+
+void ssa_set_wait_timeout_ns(uint64_t ns) {
+  std::lock_guard<std::mutex> g(ssa::g_mu);
+  ssa::g_wait_ns = ns ? (unsigned long long)ns : ssa::WAIT_TIMEOUT_NS;
 }
 
 int ssa_device_status(void* stream) {

@@ -24,7 +24,7 @@ SSA_ERR_TIMEOUT = -4
 MODE_DENSE, MODE_SKIP, MODE_NM = 0, 1, 2
 
 EXPORTED = ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
-            "ssa_device_status", "ssa_status_string", "ssa_version"]
+            "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version"]
 
 
 class SSAError(RuntimeError):
@@ -47,6 +47,8 @@ def _load():
     lib.ssa_fwd_noalloc.argtypes = fwd_args
     lib.ssa_visited_tiles.restype = ctypes.c_int64
     lib.ssa_visited_tiles.argtypes = [I, I, I, I, I]
+    lib.ssa_set_wait_timeout_ns.restype = None
+    lib.ssa_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     lib.ssa_device_status.restype = I
     lib.ssa_device_status.argtypes = [P]
     lib.ssa_status_string.restype = ctypes.c_char_p
@@ -85,6 +87,11 @@ def ssa_version() -> int:
 
 def ssa_visited_tiles(causal, Lq, Lk, Br, Bc) -> int:
     return int(lib.ssa_visited_tiles(int(causal), Lq, Lk, Br, Bc))
+
+
+def ssa_set_wait_timeout_ns(ns: int) -> None:
+    """Limit of each in-kernel pipeline wait (0 = default 2 s); a test knob."""
+    lib.ssa_set_wait_timeout_ns(int(ns))
 
 
 def ssa_device_status(stream=None) -> int:

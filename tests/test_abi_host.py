@@ -28,8 +28,8 @@ def _declared_functions():
 
 def test_header_declares_the_entry_points():
     assert _declared_functions() == sorted(
-        ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles", "ssa_device_status",
-         "ssa_status_string", "ssa_version"])
+        ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
+         "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version"])
 
 
 def test_library_exports_every_declared_symbol(ssa):
