@@ -92,7 +92,6 @@ struct __align__(8) Bars {
   uint64_t mma_done;
   uint32_t tmem_base;
   uint32_t dec_word[NQT];
-  uint32_t vote[NQT][2][4];
   uint32_t abort_flag;
 };
 
@@ -251,6 +250,66 @@ __device__ __forceinline__ void nm_select(float (&x)[64], int N, int col0, int p
   }
 }
 
+// 4-wide N:M with N fixed at compile time: the order statistics of a group
+// come from six min/max operations instead of a general sort.
+template <int NN>
+__device__ __forceinline__ void nm4_fixed(float (&x)[64], int col0, int pos, int sink, int recent,
+                                          bool windows) {
+#pragma unroll
+  for (int g = 0; g < 16; ++g) {
+    float* v = &x[4 * g];
+    const float hab = fmaxf(v[0], v[1]), lab = fminf(v[0], v[1]);
+    const float hcd = fmaxf(v[2], v[3]), lcd = fminf(v[2], v[3]);
+    const float mnh = fminf(hab, hcd), mxl = fmaxf(lab, lcd);
+    float thr, nxt;  // N-th and (N+1)-th largest
+    if constexpr (NN == 1) { thr = fmaxf(hab, hcd); nxt = fmaxf(mnh, mxl); }
+    else if constexpr (NN == 2) { thr = fmaxf(mnh, mxl); nxt = fminf(mnh, mxl); }
+    else { thr = fminf(mnh, mxl); nxt = fminf(lab, lcd); }
+    bool keep[4];
+    if (thr == nxt && thr != -INFINITY) {  // exact tie at the boundary: ranks
+      int rank[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = a + 1; c < 4; ++c) {
+          if (v[c] > v[a]) ++rank[a];
+          else ++rank[c];
+        }
+#pragma unroll
+      for (int a = 0; a < 4; ++a) keep[a] = rank[a] < NN;
+    } else {
+#pragma unroll
+      for (int a = 0; a < 4; ++a) keep[a] = v[a] >= thr;
+    }
+    if (windows) {
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const int jj = col0 + 4 * g + a;
+        const int dist = pos - jj;
+        keep[a] = keep[a] || (jj < sink) || (dist >= 0 && dist < recent);
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+      if (!keep[a]) v[a] = -INFINITY;
+  }
+}
+
+template <int M>
+__device__ __forceinline__ void nm_apply(float (&x)[64], int N, int col0, int pos, int sink,
+                                         int recent, bool windows) {
+  if constexpr (M == 4) {
+    switch (N) {  // uniform across the CTA
+      case 1: nm4_fixed<1>(x, col0, pos, sink, recent, windows); break;
+      case 2: nm4_fixed<2>(x, col0, pos, sink, recent, windows); break;
+      case 3: nm4_fixed<3>(x, col0, pos, sink, recent, windows); break;
+      default: break;  // N = 4 keeps every key
+    }
+  } else {
+    nm_select<M>(x, N, col0, pos, sink, recent, windows);
+  }
+}
+
 struct Work {
   int b, hq, hkv;
   int pt[NQT];            // 128-row tile index of tile t
@@ -335,8 +394,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
             if (jj >= p.Lk || (p.causal && jj > pos)) x[i] = -INFINITY;
           }
         }
-        if constexpr (nm_on)
-          nm_select<(NM_M ? NM_M : 4)>(x, p.n, cb, pos, p.sink, p.recent, nm_windows);
+        if constexpr (nm_on) nm_apply<(NM_M ? NM_M : 4)>(x, p.n, cb, pos, p.sink, p.recent, nm_windows);
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
         for (int i = 0; i < 64; i += 4) {
@@ -362,27 +420,29 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       }
       if (need_mask || nm_on) tmem_wait_st();
     }
+    // A warp whose wait gave up keeps going with undefined data (so every
+    // barrier and hand-off still pairs up) and keeps the tile; the failure
+    // is already recorded.
+    if (!ok && !failed && lane == 0) record_failure(p, bars);
+    if (!ok) failed = true;
     const bool negligible =
-        !valid || m_tile == -INFINITY ||
-        (m_true != -INFINITY && (m_tile - m_true) * p.scale_log2 < p.log2_lambda);
-    const uint32_t wneg = __all_sync(0xffffffffu, negligible) ? 1u : 0u;
-    if (lane == 0) bars->vote[t][j & 1][quarter] = wneg | (ok ? 0u : 2u);
-    tc_fence_before();
-    named_bar_sync(bar_vote, 128);
-    uint32_t v4[4];
-#pragma unroll
-    for (int w = 0; w < 4; ++w) v4[w] = *reinterpret_cast<volatile uint32_t*>(&bars->vote[t][j & 1][w]);
-    if ((v4[0] | v4[1] | v4[2] | v4[3]) & 2u) {
-      failed = true;
-      if (row == 0) record_failure(p, bars);
-      break;
-    }
+        ok && (!valid || m_tile == -INFINITY ||
+               (m_true != -INFINITY && (m_tile - m_true) * p.scale_log2 < p.log2_lambda));
     bool keep_h[2];
-    if (p.half) {
-      keep_h[0] = (j < nvis_h0) && !(skip_on && (v4[0] & v4[1] & 1u));
-      keep_h[1] = (j < nvis_h1) && !(skip_on && (v4[2] & v4[3] & 1u));
+    if (skip_on) {
+      // the skip vote: one barrier that ANDs "negligible" over the tile's rows
+      tc_fence_before();
+      if (p.half) {
+        const bool neg0 = bar_red_and(bar_vote, 128, half == 0 ? negligible : true);
+        const bool neg1 = bar_red_and(bar_vote, 128, half == 1 ? negligible : true);
+        keep_h[0] = (j < nvis_h0) && !neg0;
+        keep_h[1] = (j < nvis_h1) && !neg1;
+      } else {
+        keep_h[0] = keep_h[1] = !bar_red_and(bar_vote, 128, negligible);
+      }
     } else {
-      keep_h[0] = keep_h[1] = !(skip_on && (v4[0] & v4[1] & v4[2] & v4[3] & 1u));
+      keep_h[0] = j < nvis_h0;
+      keep_h[1] = j < nvis_h1;
     }
     const bool tile_keep = keep_h[0] || keep_h[1];
     const bool my_keep = half ? keep_h[1] : keep_h[0];
