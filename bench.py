@@ -22,6 +22,7 @@ import argparse
 import hashlib
 import json
 import os
+import select
 import statistics
 import subprocess
 import sys
@@ -112,9 +113,15 @@ class Clocks:
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            time.sleep(0.3)
         except OSError:
             self.proc = None
+            return self
+        # nvidia-smi's start-up can hold the driver for seconds; the timed
+        # region starts only after its first sample has arrived.
+        self.first = ""
+        ready, _, _ = select.select([self.proc.stdout], [], [], 20.0)
+        if ready:
+            self.first = self.proc.stdout.readline()
         return self
 
     def __exit__(self, *a):
@@ -123,7 +130,8 @@ class Clocks:
             time.sleep(0.1)
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                rest, _ = self.proc.communicate(timeout=5)
+                self.out = self.first + rest
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 self.out = ""
@@ -377,7 +385,7 @@ def main():
                          "peak": bf16_peak, "unit": "TFLOP/s",
                          "frac": flops_exec / (ms_step * 1e-3) / 1e12 / bf16_peak,
                          "traffic": traffic, "peak_source": f"{src} bf16 burst",
-                         "kernel": "ssa::ssa_fwd_kernel<128,128,0,0>",
+                         "kernel": f"ssa::ssa_fwd_kernel<{w.d},{w.Bc},{w.m if w.mode & 2 else 0},0>",
                          "dense_equiv_frac": flops_dense / (ms_step * 1e-3) / 1e12 / bf16_peak,
                          "hbm_frac_of_algorithmic_bytes": None},
             "gpu_launches": args.steps,

@@ -88,10 +88,11 @@ struct __align__(8) Bars {
   uint64_t q_full;
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
-  uint64_t s_full[NQT], dec_ready[NQT], dec_ack[NQT], p_ready[NQT], o_done[NQT];
+  uint64_t s_full[NQT], p_ready[NQT], o_done[NQT];
+  uint64_t vote_bar[NQT][2];  // per tile, per step parity: one arrival per softmax warp
   uint64_t mma_done;
   uint32_t tmem_base;
-  uint32_t dec_word[NQT];
+  uint32_t vote[NQT][2];      // byte w: softmax warp w of the tile keeps the key tile
   uint32_t abort_flag;
 };
 
@@ -195,118 +196,119 @@ __device__ __forceinline__ void sort_desc(float (&s)[M]) {
   }
 }
 
-// N:M selection on one thread's row (64 columns): for each aligned group of
-// M keys keep a key iff it is inside the sink / recent window or among the N
-// largest scores of its group, equal scores ranked by lower index; dropped
-// keys become -inf.  Masked keys are already -inf and stay -inf.
-// Fast path: with thr the N-th largest and nxt the (N+1)-th, thr > nxt means
-// the top N are exactly the keys >= thr (thr = -inf: every finite key).  A
-// tie (thr == nxt, finite) falls back to explicit ranks.
-template <int M>
-__device__ __forceinline__ void nm_select(float (&x)[64], int N, int col0, int pos, int sink,
-                                          int recent, bool windows) {
+// N:M selection on one thread's row, 64 columns at a time: for each aligned
+// group of M keys keep a key iff it is inside the sink / recent window or
+// among the N largest scores of its group, equal scores ranked by lower
+// index; dropped keys become -inf.  Masked keys are already -inf and stay
+// -inf.  The fast form uses thr, the N-th largest score of a group, and nxt,
+// the (N+1)-th: thr > nxt means the top N are exactly the keys >= thr
+// (thr = -inf: every finite key).  It reports whether any group had an exact
+// tie at the boundary (thr == nxt, finite); the caller then redoes the row
+// from the original scores with explicit ranks.
+// (bitwise, not short-circuit, logic throughout: the per-key decisions differ
+// between lanes and must compile to predicated selects, not branches)
+__device__ __forceinline__ bool in_window(int jj, int pos, int sink, int recent) {
+  return (jj < sink) | ((unsigned)(pos - jj) < (unsigned)recent);
+}
+
+template <bool WIN>
+__device__ __forceinline__ void nm_keep_group(float* v, int M, float thr, int col, int pos, int sink,
+                                              int recent) {
 #pragma unroll
-  for (int g = 0; g < 64 / M; ++g) {
-    float srt[M];
-#pragma unroll
-    for (int a = 0; a < M; ++a) srt[a] = x[g * M + a];
-    sort_desc<M>(srt);
-    float thr = srt[0], nxt = srt[1];
-#pragma unroll
-    for (int r = 1; r < M; ++r)
-      if (N == r + 1) {
-        thr = srt[r];
-        nxt = r + 1 < M ? srt[r + 1] : -INFINITY;
-      }
-    bool keep[M];
-    if (thr == nxt && thr != -INFINITY) {
-      int rank[M];
-#pragma unroll
-      for (int a = 0; a < M; ++a) rank[a] = 0;
-#pragma unroll
-      for (int a = 0; a < M; ++a)
-#pragma unroll
-        for (int c = a + 1; c < M; ++c) {
-          if (x[g * M + c] > x[g * M + a]) ++rank[a];
-          else ++rank[c];
-        }
-#pragma unroll
-      for (int a = 0; a < M; ++a) keep[a] = rank[a] < N;
-    } else {
-#pragma unroll
-      for (int a = 0; a < M; ++a) keep[a] = x[g * M + a] >= thr;
-    }
-    if (windows) {
-#pragma unroll
-      for (int a = 0; a < M; ++a) {
-        const int jj = col0 + g * M + a;
-        const int dist = pos - jj;
-        keep[a] = keep[a] || (jj < sink) || (dist >= 0 && dist < recent);
-      }
-    }
-#pragma unroll
-    for (int a = 0; a < M; ++a)
-      if (!keep[a]) x[g * M + a] = -INFINITY;
+  for (int a = 0; a < M; ++a) {
+    bool keep = v[a] >= thr;
+    if constexpr (WIN) keep |= in_window(col + a, pos, sink, recent);
+    v[a] = keep ? v[a] : -INFINITY;
   }
 }
 
-// 4-wide N:M with N fixed at compile time: the order statistics of a group
-// come from six min/max operations instead of a general sort.
-template <int NN>
-__device__ __forceinline__ void nm4_fixed(float (&x)[64], int col0, int pos, int sink, int recent,
-                                          bool windows) {
+// 4-wide groups, N fixed at compile time: order statistics from min/max.
+template <int NN, bool WIN>
+__device__ __forceinline__ bool nm4_fast(float (&x)[64], int col0, int pos, int sink, int recent) {
+  bool tie = false;
 #pragma unroll
   for (int g = 0; g < 16; ++g) {
     float* v = &x[4 * g];
     const float hab = fmaxf(v[0], v[1]), lab = fminf(v[0], v[1]);
     const float hcd = fmaxf(v[2], v[3]), lcd = fminf(v[2], v[3]);
     const float mnh = fminf(hab, hcd), mxl = fmaxf(lab, lcd);
-    float thr, nxt;  // N-th and (N+1)-th largest
-    if constexpr (NN == 1) { thr = fmaxf(hab, hcd); nxt = fmaxf(mnh, mxl); }
-    else if constexpr (NN == 2) { thr = fmaxf(mnh, mxl); nxt = fminf(mnh, mxl); }
-    else { thr = fminf(mnh, mxl); nxt = fminf(lab, lcd); }
-    bool keep[4];
-    if (thr == nxt && thr != -INFINITY) {  // exact tie at the boundary: ranks
-      int rank[4] = {0, 0, 0, 0};
+    float t, nx;  // N-th and (N+1)-th largest
+    if constexpr (NN == 1) { t = fmaxf(hab, hcd); nx = fmaxf(mnh, mxl); }
+    else if constexpr (NN == 2) { t = fmaxf(mnh, mxl); nx = fminf(mnh, mxl); }
+    else { t = fminf(mnh, mxl); nx = fminf(lab, lcd); }
+    tie |= (t == nx) & (t != -INFINITY);
+    nm_keep_group<WIN>(v, 4, t, col0 + 4 * g, pos, sink, recent);
+  }
+  return tie;
+}
+
+// 8-wide groups: a sorting network per group.
+template <bool WIN>
+__device__ __forceinline__ bool nm8_fast(float (&x)[64], int N, int col0, int pos, int sink, int recent) {
+  bool tie = false;
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+  for (int g = 0; g < 8; ++g) {
+    float srt[8];
 #pragma unroll
-        for (int c = a + 1; c < 4; ++c) {
-          if (v[c] > v[a]) ++rank[a];
-          else ++rank[c];
-        }
+    for (int a = 0; a < 8; ++a) srt[a] = x[8 * g + a];
+    sort_desc<8>(srt);
+    float t = srt[0], nx = srt[1];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) keep[a] = rank[a] < NN;
-    } else {
-#pragma unroll
-      for (int a = 0; a < 4; ++a) keep[a] = v[a] >= thr;
-    }
-    if (windows) {
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const int jj = col0 + 4 * g + a;
-        const int dist = pos - jj;
-        keep[a] = keep[a] || (jj < sink) || (dist >= 0 && dist < recent);
+    for (int r = 1; r < 8; ++r)
+      if (N == r + 1) {  // uniform across the CTA
+        t = srt[r];
+        nx = r + 1 < 8 ? srt[r + 1] : -INFINITY;
       }
+    tie |= (t == nx) & (t != -INFINITY);
+    nm_keep_group<WIN>(&x[8 * g], 8, t, col0 + 8 * g, pos, sink, recent);
+  }
+  return tie;
+}
+
+template <int M, bool WIN>
+__device__ __forceinline__ bool nm_fast_w(float (&x)[64], int N, int col0, int pos, int sink, int recent) {
+  if constexpr (M == 4) {
+    switch (N) {  // uniform across the CTA
+      case 1: return nm4_fast<1, WIN>(x, col0, pos, sink, recent);
+      case 2: return nm4_fast<2, WIN>(x, col0, pos, sink, recent);
+      case 3: return nm4_fast<3, WIN>(x, col0, pos, sink, recent);
+      default: return false;  // N = 4 keeps every key
     }
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-      if (!keep[a]) v[a] = -INFINITY;
+  } else {
+    return nm8_fast<WIN>(x, N, col0, pos, sink, recent);
   }
 }
 
 template <int M>
-__device__ __forceinline__ void nm_apply(float (&x)[64], int N, int col0, int pos, int sink,
-                                         int recent, bool windows) {
-  if constexpr (M == 4) {
-    switch (N) {  // uniform across the CTA
-      case 1: nm4_fixed<1>(x, col0, pos, sink, recent, windows); break;
-      case 2: nm4_fixed<2>(x, col0, pos, sink, recent, windows); break;
-      case 3: nm4_fixed<3>(x, col0, pos, sink, recent, windows); break;
-      default: break;  // N = 4 keeps every key
+__device__ __forceinline__ bool nm_fast(float (&x)[64], int N, int col0, int pos, int sink, int recent,
+                                        bool windows) {
+  // windows is uniform across the CTA for a key tile
+  return windows ? nm_fast_w<M, true>(x, N, col0, pos, sink, recent)
+                 : nm_fast_w<M, false>(x, N, col0, pos, sink, recent);
+}
+
+// Explicit ranks (the exact-tie path): rank = number of group keys that
+// come first, a higher score or an equal score at a lower index.
+template <int M>
+__device__ __forceinline__ void nm_by_rank(float (&x)[64], int N, int col0, int pos, int sink,
+                                           int recent, bool windows) {
+#pragma unroll
+  for (int g = 0; g < 64 / M; ++g) {
+    int rank[M];
+#pragma unroll
+    for (int a = 0; a < M; ++a) rank[a] = 0;
+#pragma unroll
+    for (int a = 0; a < M; ++a)
+#pragma unroll
+      for (int c = a + 1; c < M; ++c) {
+        if (x[g * M + c] > x[g * M + a]) ++rank[a];
+        else ++rank[c];
+      }
+#pragma unroll
+    for (int a = 0; a < M; ++a) {
+      const bool keep = (rank[a] < N) | (windows & in_window(col0 + g * M + a, pos, sink, recent));
+      x[g * M + a] = keep ? x[g * M + a] : -INFINITY;
     }
-  } else {
-    nm_select<M>(x, N, col0, pos, sink, recent, windows);
   }
 }
 
@@ -337,7 +339,9 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
   const bool leader = p.half ? ((row & 63) == 0) : (row == 0);
   const int my_nvis = half ? nvis_h1 : nvis_h0;
   const int nvis = nvis_h0 > nvis_h1 ? nvis_h0 : nvis_h1;
-  const uint32_t bar_vote = 1 + t;
+  // speculative exponentials are exact only while a skipped tile cannot raise the max
+  const bool spec_ok = p.log2_lambda <= 0.f;
+  bool prev_keep = true;
 
   float m_true = -INFINITY;  // running max over kept tiles (raw q.k units)
   float m_ref = -INFINITY;   // reference the O accumulator and l are scaled to
@@ -352,73 +356,72 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     ok = __all_sync(0xffffffffu, ok);
     float m_tile = -INFINITY;
     const int col0 = j * BC;
-    // Pass 1, 64 columns at a time: masks, N:M, tile row max.  Masked
-    // scores are written back to TMEM so pass 2 needs no mask.
+    // Pass 1: the whole row of S in registers -- masks, N:M, tile row max.
+    // The scores stay in registers through the vote and become P in pass 2.
     const bool need_mask = (col0 + BC > p.Lk) || (p.causal && col0 + BC - 1 > pos_first);
     // does this key tile meet the sink or any row's recent window?
     const bool nm_windows = nm_on && ((col0 < p.sink) ||
                                       (col0 <= pos_first + BM - 1 && col0 + BC - 1 > pos_first - p.recent));
-    if (ok && !nm_on && !need_mask) {
-      // common case: one TMEM round trip for the whole row, max only
-      tc_fence_after();
-      float xa[BC];
+    float x[BC];
+    // S from TMEM with the causal / length mask applied
+    auto load_scores = [&]() {
 #pragma unroll
-      for (int c = 0; c < BC / 32; ++c) tmem_ld32f(lane_base + s_col + 32 * c, &xa[32 * c]);
+      for (int c = 0; c < BC / 32; ++c) tmem_ld32f(lane_base + s_col + 32 * c, &x[32 * c]);
       tmem_wait_ld();
-      float mx0 = -INFINITY, mx1 = -INFINITY;
+      if (need_mask) {
+        // last visible column of this row, relative to the tile
+        int lim = p.Lk - 1 - col0;
+        if (p.causal && pos - col0 < lim) lim = pos - col0;
 #pragma unroll
-      for (int i = 0; i < BC; i += 4) {
-        mx0 = fmax3(mx0, xa[i], xa[i + 1]);
-        mx1 = fmax3(mx1, xa[i + 2], xa[i + 3]);
+        for (int i = 0; i < BC; ++i)
+          if (i > lim) x[i] = -INFINITY;
       }
-      m_tile = fmax3(m_tile, mx0, mx1);
+    };
+    if (ok) {
+      tc_fence_after();
+      load_scores();
+      if constexpr (nm_on) {
+        constexpr int MM = NM_M ? NM_M : 4;
+        bool tie = false;
+#pragma unroll
+        for (int bb = 0; bb < BC / 64; ++bb)
+          tie |= nm_fast<MM>(*reinterpret_cast<float(*)[64]>(&x[64 * bb]), p.n, col0 + 64 * bb, pos,
+                             p.sink, p.recent, nm_windows);
+        if (__any_sync(0xffffffffu, tie)) {
+          // an exact tie at a group boundary in some row of this warp: the
+          // whole warp starts again from the scores (still in TMEM; the
+          // tcgen05 load is warp-collective) and ranks explicitly
+          load_scores();
+#pragma unroll
+          for (int bb = 0; bb < BC / 64; ++bb)
+            nm_by_rank<MM>(*reinterpret_cast<float(*)[64]>(&x[64 * bb]), p.n, col0 + 64 * bb, pos,
+                           p.sink, p.recent, nm_windows);
+        }
+      }
+      // four independent chains keep the dependent depth at BC / 8
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < BC; i += 8) {
+        mx0 = fmax3(mx0, x[i], x[i + 1]);
+        mx1 = fmax3(mx1, x[i + 2], x[i + 3]);
+        mx2 = fmax3(mx2, x[i + 4], x[i + 5]);
+        mx3 = fmax3(mx3, x[i + 6], x[i + 7]);
+      }
+      m_tile = fmaxf(fmax3(mx0, mx1, mx2), mx3);
       if (DBG && p.keep_bits != nullptr && valid && j < my_nvis) {
         uint32_t* kb = p.keep_bits + ((size_t)(b * p.Hq + hq) * p.Lq + grow) * p.Lkw;
 #pragma unroll
-        for (int w = 0; w < BC / 32; ++w) kb[col0 / 32 + w] = 0xffffffffu;
-      }
-    } else if (ok) {
-      tc_fence_after();
-#pragma unroll 1
-      for (int bb = 0; bb < BC / 64; ++bb) {
-        float x[64];
-        const uint32_t ta = lane_base + s_col + 64 * bb;
-        tmem_ld32f(ta, &x[0]);
-        tmem_ld32f(ta + 32, &x[32]);
-        tmem_wait_ld();
-        const int cb = col0 + 64 * bb;
-        if (need_mask) {
+        for (int w = 0; w < BC / 32; ++w) {
+          uint32_t word = 0;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const int jj = cb + i;
-            if (jj >= p.Lk || (p.causal && jj > pos)) x[i] = -INFINITY;
-          }
-        }
-        if constexpr (nm_on) nm_apply<(NM_M ? NM_M : 4)>(x, p.n, cb, pos, p.sink, p.recent, nm_windows);
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 64; i += 4) {
-          mx0 = fmax3(mx0, x[i], x[i + 1]);
-          mx1 = fmax3(mx1, x[i + 2], x[i + 3]);
-        }
-        m_tile = fmax3(m_tile, mx0, mx1);
-        if (need_mask || nm_on) {
-          tmem_st32(ta, *reinterpret_cast<const uint32_t(*)[32]>(&x[0]));
-          tmem_st32(ta + 32, *reinterpret_cast<const uint32_t(*)[32]>(&x[32]));
-        }
-        if (DBG && p.keep_bits != nullptr && valid && j < my_nvis) {
-          uint32_t* kb = p.keep_bits + ((size_t)(b * p.Hq + hq) * p.Lq + grow) * p.Lkw;
-#pragma unroll
-          for (int w = 0; w < 2; ++w) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int u = 0; u < 32; ++u) word |= (x[32 * w + u] != -INFINITY ? 1u : 0u) << u;
-            const int wi = cb / 32 + w;
-            if (wi < p.Lkw) kb[wi] = word;
-          }
+          for (int u = 0; u < 32; ++u) word |= (x[32 * w + u] != -INFINITY ? 1u : 0u) << u;
+          const int wi = col0 / 32 + w;
+          if (wi < p.Lkw) kb[wi] = word;
         }
       }
-      if (need_mask || nm_on) tmem_wait_st();
+    } else {
+#pragma unroll
+      for (int i = 0; i < BC; ++i) x[i] = -INFINITY;
     }
     // A warp whose wait gave up keeps going with undefined data (so every
     // barrier and hand-off still pairs up) and keeps the tile; the failure
@@ -428,74 +431,58 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     const bool negligible =
         ok && (!valid || m_tile == -INFINITY ||
                (m_true != -INFINITY && (m_tile - m_true) * p.scale_log2 < p.log2_lambda));
-    bool keep_h[2];
+    // The skip vote: each warp publishes one byte, "some row of mine keeps
+    // the tile", and arrives on the tile's vote barrier for this step's
+    // parity.  The MMA warp and the V producer read the same four bytes.
+    const uint32_t vbar = smem_u32(&bars->vote_bar[t][j & 1]);
     if (skip_on) {
-      // the skip vote: one barrier that ANDs "negligible" over the tile's rows
-      tc_fence_before();
-      if (p.half) {
-        const bool neg0 = bar_red_and(bar_vote, 128, half == 0 ? negligible : true);
-        const bool neg1 = bar_red_and(bar_vote, 128, half == 1 ? negligible : true);
-        keep_h[0] = (j < nvis_h0) && !neg0;
-        keep_h[1] = (j < nvis_h1) && !neg1;
-      } else {
-        keep_h[0] = keep_h[1] = !bar_red_and(bar_vote, 128, negligible);
-      }
-    } else {
-      keep_h[0] = j < nvis_h0;
-      keep_h[1] = j < nvis_h1;
-    }
-    const bool tile_keep = keep_h[0] || keep_h[1];
-    const bool my_keep = half ? keep_h[1] : keep_h[0];
-    if (leader && j < my_nvis) {
-      if (!my_keep) {
-        ++skipped;
-        skip_word |= 1u << (j & 31);
-      }
-      if (DBG && p.skip_bits != nullptr && ((j & 31) == 31 || j == my_nvis - 1)) {
-        const int qt = p.half ? 2 * pt + half : pt;
-        p.skip_bits[((size_t)(b * p.Hq + hq) * p.nQ + qt) * p.nKw + (j >> 5)] = skip_word;
-        skip_word = 0;
+      const bool wkeep = !__all_sync(0xffffffffu, negligible) && j < my_nvis;
+      if (lane == 0) {
+        st_shared_u8(smem_u32(&bars->vote[t][j & 1]) + quarter, wkeep ? 1u : 0u);
+        mbar_arrive(vbar);
       }
     }
-    if (row == 0) {
-      // the V producer must have taken decision j-1 before decision j is
-      // published on the same barrier (keeps its phases from aliasing)
-      if (j > 0 && !mbar_wait_fast(smem_u32(&bars->dec_ack[t]), (j - 1) & 1, p.wait_ns))
-        record_failure(p, bars);
-      bars->dec_word[t] = tile_keep ? 1u : 0u;
-      mbar_arrive(smem_u32(&bars->dec_ready[t]));
+    bool keep_h[2] = {j < nvis_h0, j < nvis_h1};
+    // (warp-uniform outcome: the tcgen05 accesses that follow are warp-collective)
+    auto decide = [&]() {
+      if (!__all_sync(0xffffffffu, mbar_wait(vbar, (j >> 1) & 1, p.wait_ns))) {
+        if (!failed && lane == 0) record_failure(p, bars);
+        failed = true;
+        return;  // keep the tile
+      }
+      const uint32_t w = ld_shared_u32(smem_u32(&bars->vote[t][j & 1]));
+      keep_h[0] = p.half ? (w & 0xffffu) != 0u : w != 0u;
+      keep_h[1] = p.half ? (w >> 16) != 0u : w != 0u;
+    };
+    // With lambda <= 1 a tile that ends up skipped has every row's max below
+    // the running max, so computing its P against the updated max changes
+    // nothing: the exponentials may start before the vote completes.  A
+    // tile right after a skipped one waits for the vote instead, so long
+    // runs of skipped tiles spend no MUFU time.
+    bool decided = !skip_on;
+    if (!decided && !(spec_ok && prev_keep)) {
+      decide();
+      decided = true;
     }
-    if (!tile_keep) {
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[t]));
-      continue;
-    }
-
-    if (my_keep) {
-      m_true = fmaxf(m_true, m_tile);
+    if (!decided || (half ? keep_h[1] : keep_h[0])) {
+      const float m_new = fmaxf(m_true, m_tile);
       bool resc = false;
-      if (m_ref == -INFINITY) m_ref = m_true;  // first kept key: O and l are still zero
-      else resc = (m_true - m_ref) * p.scale_log2 > RESCALE_LOG2;
+      float m_ref_new = m_ref, alpha = 1.f;
+      if (m_ref == -INFINITY) m_ref_new = m_new;  // first kept key: O and l are still zero
+      else resc = (m_new - m_ref) * p.scale_log2 > RESCALE_LOG2;
       // O is rescaled after P is written (the S registers are free then);
       // every earlier P.V of this tile completed before S(j) did.
       const bool any_resc = __any_sync(0xffffffffu, resc);
-      float alpha = 1.f;
       if (resc) {
-        alpha = mufu_exp2((m_ref - m_true) * p.scale_log2);
-        l *= alpha;
-        m_ref = m_true;
+        alpha = mufu_exp2((m_ref - m_new) * p.scale_log2);
+        m_ref_new = m_new;
       }
-      // Pass 2: P = exp2((s - m_ref) * scale * log2 e), 64 columns at a time
+      // Pass 2: P = exp2((s - m_ref) * scale * log2 e) from the registers
+      // pass 1 left, 32 bf16 pairs per 64 columns
       const float c = p.scale_log2;
-      const float mref_s = (m_ref == -INFINITY) ? 0.f : m_ref * c;
+      const float mref_s = (m_ref_new == -INFINITY) ? 0.f : m_ref_new * c;
       const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-mref_s, -mref_s);
       uint64_t ls2 = f2_pack(0.f, 0.f);
-      // all of S in one TMEM round trip, then 32 bf16 pairs per 64 columns
-      float x[BC];
-#pragma unroll
-      for (int cc = 0; cc < BC / 32; ++cc) tmem_ld32f(lane_base + s_col + 32 * cc, &x[32 * cc]);
-      tmem_wait_ld();
 #pragma unroll
       for (int bb = 0; bb < BC / 64; ++bb) {
         uint32_t pk[32];
@@ -518,32 +505,62 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
         }
         tmem_st32(lane_base + s_col + 32 * bb, pk);
       }
-      float ls0, ls1;
-      f2_unpack(ls2, ls0, ls1);
-      l += ls0 + ls1;
-      if (any_resc && n_pv > 0) {
+      if (!decided) decide();
+      const bool mine = half ? keep_h[1] : keep_h[0];
+      if (mine) {
+        float ls0, ls1;
+        f2_unpack(ls2, ls0, ls1);
+        l = l * alpha + (ls0 + ls1);
+        m_true = m_new;
+        m_ref = m_ref_new;
+        if (any_resc && n_pv > 0) {
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + o_col + 32 * c, o);
-          tmem_wait_ld();
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + o_col + 32 * cc, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(lane_base + o_col + 32 * c, o);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(lane_base + o_col + 32 * cc, o);
+          }
         }
+      } else if (keep_h[0] || keep_h[1]) {
+        // speculated, and only the other half of a 64-row pair keeps it
+        tmem_wait_st();
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
+#pragma unroll
+        for (int h = 0; h < BC / 64; ++h) tmem_st32(lane_base + s_col + 32 * h, pk);
       }
-    } else {
+    } else if (keep_h[0] || keep_h[1]) {
+      // decided: only the other half of a 64-row pair keeps this key tile
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) pk[i] = 0u;
 #pragma unroll
       for (int h = 0; h < BC / 64; ++h) tmem_st32(lane_base + s_col + 32 * h, pk);
     }
+    const bool tile_keep = keep_h[0] || keep_h[1];
+    const bool my_keep = half ? keep_h[1] : keep_h[0];
+    prev_keep = tile_keep;
+    if (leader && j < my_nvis) {
+      if (!my_keep) {
+        ++skipped;
+        skip_word |= 1u << (j & 31);
+      }
+      if (DBG && p.skip_bits != nullptr && ((j & 31) == 31 || j == my_nvis - 1)) {
+        const int qt = p.half ? 2 * pt + half : pt;
+        p.skip_bits[((size_t)(b * p.Hq + hq) * p.nQ + qt) * p.nKw + (j >> 5)] = skip_word;
+        skip_word = 0;
+      }
+    }
+    // P (or nothing, for a skipped tile) is in TMEM: hand the step to the MMA warp
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&bars->p_ready[t]));
-    ++n_pv;
+    if (tile_keep) ++n_pv;
   }
 
   // ---- epilogue
@@ -605,6 +622,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t v_s = smem_u32(smem + L::V_OFF);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool skip_on = (p.mode & SSA_MODE_SKIP) != 0;
 
   // ---- work item: heaviest causal pairs first; query heads that share a KV
   // head are adjacent in launch order.
@@ -650,8 +668,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int i = 0; i < NQT; ++i) {
       mbar_init(smem_u32(&bars->s_full[i]), 1);
-      mbar_init(smem_u32(&bars->dec_ready[i]), 1);
-      mbar_init(smem_u32(&bars->dec_ack[i]), 1);
+      mbar_init(smem_u32(&bars->vote_bar[i][0]), 4);
+      mbar_init(smem_u32(&bars->vote_bar[i][1]), 4);
       mbar_init(smem_u32(&bars->p_ready[i]), 4);  // one arrival per softmax warp
       mbar_init(smem_u32(&bars->o_done[i]), 1);
     }
@@ -724,12 +742,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
           if (j >= wk.nvis_t[t]) continue;
-          if (!mbar_wait_fast(smem_u32(&bars->dec_ready[t]), j & 1, p.wait_ns)) {
-            fail = true;
-            break;
+          bool keep = true;
+          if (skip_on) {
+            if (!mbar_wait_fast(smem_u32(&bars->vote_bar[t][j & 1]), (j >> 1) & 1, p.wait_ns)) {
+              fail = true;
+              break;
+            }
+            keep = ld_shared_u32(smem_u32(&bars->vote[t][j & 1])) != 0u;
           }
-          const uint32_t keep = *reinterpret_cast<volatile uint32_t*>(&bars->dec_word[t]);
-          mbar_arrive(smem_u32(&bars->dec_ack[t]));
           if (keep && !loaded) {
             mbar_arrive_expect_tx(fb, L::V_BYTES);
 #pragma unroll
@@ -798,7 +818,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int t = 0; t < NQT; ++t) {
           if (j >= wk.nvis_t[t]) continue;
           if (!mbar_wait_fast(smem_u32(&bars->p_ready[t]), j & 1, p.wait_ns)) { ok = false; break; }
-          const uint32_t keep = *reinterpret_cast<volatile uint32_t*>(&bars->dec_word[t]);
+          const bool keep = !skip_on || ld_shared_u32(smem_u32(&bars->vote[t][j & 1])) != 0u;
           if (keep) {
             if (!v_seen) {
               if (!mbar_wait_fast(smem_u32(&bars->v_full[slot]), (j / VST) & 1, p.wait_ns)) { ok = false; break; }
