@@ -201,18 +201,158 @@ def run_reference(args, w, lam, rank, world):
     per_step = []
     info = None
     for s in range(min(args.warmup, 1)):
-        cpu_baseline(w, lam, 0.0, seed=99)
+        (decode_cpu_baseline if w.Lq else cpu_baseline)(w, lam, 0.0, seed=99)
     for s in range(max(1, args.steps)):
-        info = cpu_baseline(w, lam, 0.0, seed=100 + s)
+        info = (decode_cpu_baseline(w, lam, 0.0, seed=100 + s) if w.Lq
+                else cpu_baseline(w, lam, 0.0, seed=100 + s))
         per_step.append(info["value"])
     val = statistics.median(per_step)
-    line = {"impl": "reference", "metric": "attn fwd TFLOP/s (dense-equiv)", "value": val,
-            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+    metric = "attn decode HBM GB/s (K, V, Q, O, lse once)" if w.Lq else "attn fwd TFLOP/s (dense-equiv)"
+    line = {"impl": "reference", "metric": metric, "value": val,
+            "unit": info["unit"], "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": workload_name(w, lam)},
             "cpu_baseline": dict(info, value=val),
-            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "e2e": {"value": val, "unit": info["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def decode_cpu_baseline(w, lam, budget_s: float, seed: int = 7):
+    """The fp64 decode oracle (numpy) on a bounded sample of (sequence, head)
+    pairs of the decode workload; dense-equivalent FLOPs of the sample / wall."""
+    from oracle.decode import decode as decode_oracle
+    q, k, v = make_inputs(w, "cpu")
+    g = torch.Generator().manual_seed(seed)
+    done, t_total = 0, 0.0
+    while done == 0 or t_total < budget_s:
+        heads = [(int(torch.randint(w.B, (1,), generator=g)), int(torch.randint(w.Hq, (1,), generator=g)))]
+        t0 = time.perf_counter()
+        decode_oracle(q, k, v, causal=w.causal, scale=w.scale, lam=lam, Bc=w.Bc, num_splits=w.splits,
+                      heads=heads)
+        t_total += time.perf_counter() - t0
+        done += 1
+    per_head = decode_alg_bytes(w) / (w.B * w.Hq)
+    return {"value": per_head * done / t_total / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} random (sequence, head) pairs of {w.name} (lambda={lam:g}), fp64 numpy "
+                      f"decode oracle, {t_total:.1f} s wall; the pairs' share of the algorithmic bytes / wall"}
+
+
+def decode_alg_bytes(w) -> float:
+    """K and V read once, Q and O (bf16) and lse (fp32) once."""
+    return 2.0 * w.B * w.L * w.Hkv * w.d * 2 + 2.0 * 2 * w.B * w.Lq * w.Hq * w.d + 4.0 * w.B * w.Hq * w.Lq
+
+
+def run_decode(args, w, lam, rank, world, local_rank):
+    """Decode leg: ssa_decode on a resident KV cache.  HBM-bound, so the
+    roofline is bytes: K and V read once, Q, O and lse once."""
+    import torch.distributed as tdist
+    dist = None
+    if world > 1:
+        import datetime
+        dist = tdist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    from softmax_ssa_fwd_b200 import ssa
+    dev = torch.device("cuda", local_rank)
+    nK = -(-w.L // w.Bc)
+    ws_bytes = ssa.ssa_decode_workspace_bytes(w.B, w.Hq, w.Lq, w.d, w.splits)
+    sets = []
+    for s in range(2):  # two KV caches of 1.07 GB each, alternated: > 126 MB L2
+        q, k, v = make_inputs(w.with_(seed=w.seed + 1000 * s + 17 * rank), dev)
+        out = torch.empty_like(q)
+        lse = torch.empty(w.B, w.Hq, w.Lq, dtype=torch.float32, device=dev)
+        cnt = torch.empty(w.B, w.Hq, dtype=torch.int32, device=dev)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        sets.append((q, k, v, out, lse, cnt, ws))
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, qq=None):
+        q, k, v, out, lse, cnt, ws = sets[i & 1]
+        st = ssa.ssa_decode(q if qq is None else qq, k, v, out, lse, cnt, w.B, w.Hq, w.Hkv, w.Lq, w.L,
+                            w.d, w.causal, w.scale, lam, w.Bc, w.splits, ws, ws_bytes, stream)
+        if st != 0:
+            raise RuntimeError(ssa.status_string(st))
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local_rank) as clk:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        e1.synchronize()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+    ms_step = reduce_max(e0.elapsed_time(e1), dist, dev) / args.steps
+    skipped = float(sets[(args.steps - 1) & 1][5].sum().item())
+    visited = float(w.B * w.Hq * nK)
+    bf16_peak, _, hbm_peak, src = peaks()
+    alg_bytes = decode_alg_bytes(w)
+    flops = dense_equiv_flops(w, Lq=w.Lq)
+    gbs = job_rate(alg_bytes, world, ms_step) / 1e9
+    # e2e: the step's new query rows from pinned host memory, out + lse + counts back
+    e2e = None
+    if not args.no_e2e:
+        q, k, v, out, lse, cnt, ws = sets[0]
+        hq_ = q.cpu().pin_memory()
+        ho, hl, hc = (torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (out, lse, cnt))
+        dq = torch.empty_like(q)
+        n_e2e = max(3, min(args.steps, 50))
+
+        def e2e_step():
+            dq.copy_(hq_, non_blocking=True)
+            step(0, dq)
+            ho.copy_(out, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+            hc.copy_(cnt, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        e1.synchronize()
+        ems = reduce_max(e0.elapsed_time(e1), dist, dev) / n_e2e
+        e2e = {"value": job_rate(alg_bytes, world, ems) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": hq_.numel() * hq_.element_size(),
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in (ho, hl, hc)),
+               "ms_per_step": ems, "steps": n_e2e, "kv_cache": "resident on the GPU (decode state)"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = decode_cpu_baseline(w, lam, args.cpu_budget)
+    if rank == 0:
+        line = {
+            "metric": "attn decode HBM GB/s (K, V, Q, O, lse once)", "value": gbs, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": workload_name(w, lam) + f" decode Lq={w.Lq} splits={w.splits}",
+                       "parallelism": f"replicas x{world}",
+                       "l2": "two KV caches of 1.07 GB alternated (> 126 MB L2)"},
+            "dense_equiv_tflops": job_rate(flops, world, ms_step) / 1e12,
+            "tiles_skipped_frac": skipped / visited, "tiles_visited": visited, "tiles_skipped": skipped,
+            "tokens_per_s": job_rate(w.B * w.Lq, world, ms_step),
+            "roofline": {"bound": "hbm", "achieved": gbs / world, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": gbs / world / hbm_peak, "traffic": None,
+                         "peak_source": f"{src} HBM copy",
+                         "kernel": "ssa_dec::decode_split_kernel + decode_combine_kernel",
+                         "algorithmic_bytes": alg_bytes},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk.summary(), "e2e": e2e, "cpu_baseline": cpu, "kernel_hash": kernel_hash(),
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
     return 0
 
 
@@ -243,7 +383,7 @@ def main():
         if w.rope == "3d":
             raise SystemExit("--L does not apply to the 3D-rotary video workload")
         w = w.with_(L=args.L, name=f"{w.name}@L{args.L}")
-    lam = args.lam if args.lam is not None else (1e-3 if w.mode & MODE_SKIP else 0.0)
+    lam = args.lam if args.lam is not None else (w.lambdas[0] if w.Lq else (1e-3 if w.mode & MODE_SKIP else 0.0))
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -251,6 +391,9 @@ def main():
 
     if args.impl == "reference":
         return run_reference(args, w, lam, rank, world)
+    if w.Lq:
+        torch.cuda.set_device(local_rank)
+        return run_decode(args, w, lam, rank, world, local_rank)
 
     torch.cuda.set_device(local_rank)
     dist = None

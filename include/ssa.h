@@ -52,6 +52,7 @@
 #ifndef SSA_H
 #define SSA_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -137,6 +138,43 @@ void ssa_set_wait_timeout_ns(uint64_t ns);
  * device recorded a timed-out wait since the last call, and clears the word.
  * Returns SSA_ERR_CUDA if the synchronisation itself fails. */
 int ssa_device_status(void* stream);
+
+/* Decode-phase skip-softmax attention: a few query rows per sequence (Lq,
+ * e.g. 1 new token, or a handful of speculative ones) against a long KV cache.
+ * "Attention Sparsity for HuggingFace Models" (custom configuration) gives
+ * skip-softmax separate prefill and decode thresholds; N:M is prefill only,
+ * so there is no N:M here.  Layouts, GQA mapping, the bottom-right causal
+ * mask, scale and lambda are those of ssa_fwd; the query tile is the Lq rows
+ * of one query head (Lq <= Br), so a key tile is skipped for a head when
+ * exp(tile_row_max - running_max) < lambda for each of its rows.
+ *
+ * The key tiles of each sequence are split into num_splits contiguous ranges
+ * of ceil(nK / num_splits) tiles, nK = ceil(Lk / Bc), processed in parallel.
+ * Each range runs the skip-softmax recurrence with its OWN running max (its
+ * first tile is never skipped unless fully masked), and the ranges are merged
+ * by the log-sum-exp rule.  With num_splits == 1 this is exactly ssa_fwd's
+ * rule for one query tile; with more splits it is this reading of the method
+ * for split-KV decoding (the pages do not define one), and skip decisions can
+ * differ from the single-range ones.
+ *
+ *   tile_skip_count: [B, Hq] int32, skipped key tiles per (batch, head),
+ *                    summed over splits (overwritten).
+ *   workspace:       device scratch of at least ssa_decode_workspace_bytes()
+ *                    bytes, 16-byte aligned, owned by the caller; holds the
+ *                    per-split partial results between the two kernels.
+ *   Limits: d in {64, 128}, Bc in {64, 128}, (Hq / Hkv) * Lq <= 32
+ *   (SSA_ERR_UNSUPPORTED otherwise); num_splits >= 1 (splits past the last
+ *   key tile are empty and harmless).
+ * Two kernels are enqueued on `stream`; no device memory is allocated.
+ * Returns SSA_OK once enqueued, SSA_ERR_INVALID_ARG / SSA_ERR_UNSUPPORTED
+ * (nothing enqueued) or SSA_ERR_CUDA. */
+int ssa_decode(const void* q, const void* k, const void* v, void* out, float* lse,
+               int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
+               float scale, float lambda, int Bc, int num_splits, void* workspace,
+               size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace ssa_decode needs for this shape (0 for invalid sizes). */
+size_t ssa_decode_workspace_bytes(int B, int Hq, int Lq, int d, int num_splits);
 
 /* Human-readable name of a status code (static storage). */
 const char* ssa_status_string(int status);

@@ -18,6 +18,10 @@ Workloads (shapes from the pages' targets: Llama-3.1-8B / Qwen3-8B prefill in
                   3D RoPE over (t, h, w), seed 3, lambda = 1e-3
 * ``qwen32k``     B=2 Hq=32 Hkv=8 L=32768 d=128 causal, RoPE base 1e6, seed 4,
                   skip + N:M 2:4 (sink 4, recent 128), lambda = 1e-3
+* ``qwen32k_decode``  decode: B=8 sequences, one new query row each (the last
+                  position) against L=32768 cached keys, Hq=32 Hkv=8 d=128,
+                  RoPE base 1e6, seed 5, lambda = 1e-4 (the pages' decode
+                  threshold), 16 key splits
 
 Recipe: one torch.Generator per workload seeded as listed.  Draw u ~ N(0, I_d)
 and normalise it (a unit "sink direction" shared by every head), then Q, K, V
@@ -66,6 +70,8 @@ class Workload:
     sink_coef: float = 3.0      # coefficient of the shared unit direction u
     local_alpha: float = 0.0    # per-head shared pre-rotary vector (3d only)
     grid: tuple = ()            # (T, H, W) for the 3d rotary embedding
+    Lq: int = 0                 # decode: query rows (the last Lq positions); 0 = L (prefill)
+    splits: int = 0             # decode: key splits
 
     @property
     def scale(self) -> float:
@@ -88,6 +94,10 @@ WORKLOADS = {
                     rope="3d", rope_base=1e4, sink_coef=0.0, grid=(21, 45, 80)),
     "qwen32k": Workload("qwen32k", 2, 32, 8, 32768, 128, True, 128, 128, MODE_SKIP | MODE_NM,
                         (1e-3,), n=2, m=4, sink=4, recent=128, seed=4, rope="1d", rope_base=1e6),
+    # decode phase: one new token per sequence against a 32k cache, 8 sequences,
+    # the pages' decode threshold 1e-4; no N:M (prefill only)
+    "qwen32k_decode": Workload("qwen32k_decode", 8, 32, 8, 32768, 128, True, 128, 128, MODE_SKIP,
+                               (1e-4,), seed=5, rope="1d", rope_base=1e6, Lq=1, splits=16),
 }
 
 
@@ -123,14 +133,16 @@ def _angles_3d(grid, d: int, base: float, device) -> torch.Tensor:
 
 
 def make_inputs(w: Workload, device="cpu"):
-    """Return (q, k, v) bf16 tensors: q [B, L, Hq, d], k and v [B, L, Hkv, d]."""
+    """Return (q, k, v) bf16 tensors: q [B, Lq, Hq, d] (Lq = L unless the
+    workload is a decode one), k and v [B, L, Hkv, d]."""
     dev = torch.device(device)
     g = torch.Generator(device=dev)
     g.manual_seed(w.seed)
     B, L, d = w.B, w.L, w.d
     u = torch.randn(d, generator=g, device=dev, dtype=torch.float32)
     u = u / u.norm()
-    q = torch.randn(B, L, w.Hq, d, generator=g, device=dev, dtype=torch.float32)
+    Lq = w.Lq if 0 < w.Lq < L else L  # decode: queries at the last Lq positions
+    q = torch.randn(B, Lq, w.Hq, d, generator=g, device=dev, dtype=torch.float32)
     k = torch.randn(B, L, w.Hkv, d, generator=g, device=dev, dtype=torch.float32)
     v = torch.randn(B, L, w.Hkv, d, generator=g, device=dev, dtype=torch.float32)
     if w.local_alpha:
@@ -139,10 +151,10 @@ def make_inputs(w: Workload, device="cpu"):
         k += w.local_alpha * a[None, None]
     if w.rope == "1d":
         ang = _angles_1d(L, d, w.rope_base, dev)
-        q, k = _rotate(q, ang), _rotate(k, ang)
+        q, k = _rotate(q, ang[L - Lq:]), _rotate(k, ang)
     elif w.rope == "3d":
         ang = _angles_3d(w.grid, d, w.rope_base, dev)
-        q, k = _rotate(q, ang), _rotate(k, ang)
+        q, k = _rotate(q, ang[L - Lq:]), _rotate(k, ang)
     if w.sink_coef:
         q += w.sink_coef * u
         k[:, :4] += w.sink_coef * u

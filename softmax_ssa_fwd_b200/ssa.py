@@ -24,7 +24,8 @@ SSA_ERR_TIMEOUT = -4
 MODE_DENSE, MODE_SKIP, MODE_NM = 0, 1, 2
 
 EXPORTED = ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
-            "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version"]
+            "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version",
+            "ssa_decode", "ssa_decode_workspace_bytes"]
 
 
 class SSAError(RuntimeError):
@@ -55,6 +56,10 @@ def _load():
     lib.ssa_status_string.argtypes = [I]
     lib.ssa_version.restype = I
     lib.ssa_version.argtypes = []
+    lib.ssa_decode.restype = I
+    lib.ssa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, F, I, I, P, ctypes.c_size_t, P]
+    lib.ssa_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.ssa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
     return lib
 
 
@@ -150,4 +155,48 @@ def attention(q, k, v, *, causal=True, scale=None, mode=MODE_SKIP, lam=0.0, n=0,
                            lam, n, m, sink, recent, Br, Bc, stream, skip_bits, keep_bits)
     if st != SSA_OK:
         raise SSAError(st, "ssa_fwd")
+    return out, lse, counts
+
+
+def ssa_decode_workspace_bytes(B, Hq, Lq, d, num_splits) -> int:
+    return int(lib.ssa_decode_workspace_bytes(B, Hq, Lq, d, num_splits))
+
+
+def ssa_decode(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, lam, Bc,
+               num_splits, workspace, workspace_bytes, stream=None) -> int:
+    """Direct call of the decode entry point; returns its status code."""
+    return lib.ssa_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(tile_skip_count),
+                          B, Hq, Hkv, Lq, Lk, d, int(causal), float(scale), float(lam), Bc,
+                          num_splits, _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def decode(q, k, v, *, causal=True, scale=None, lam=0.0, Bc=128, num_splits=None, stream=None,
+           out=None, lse=None, counts=None, workspace=None):
+    """Decode-phase skip-softmax attention through the C ABI (torch allocates).
+
+    q [B, Lq, Hq, d] (a few rows), k/v [B, Lk, Hkv, d] bf16 CUDA tensors.  Returns
+    (out [B, Lq, Hq, d] bf16, lse [B, Hq, Lq] fp32, tile_skip_count [B, Hq] int32).
+    num_splits defaults to enough key splits for about two CTAs per SM.
+    """
+    B, Lq, Hq, d = q.shape
+    _, Lk, Hkv, _ = k.shape
+    if scale is None:
+        scale = d ** -0.5
+    nK = -(-Lk // Bc)
+    if num_splits is None:
+        sms = torch.cuda.get_device_properties(q.device).multi_processor_count
+        num_splits = max(1, min(nK, -(-2 * sms // (B * Hkv))))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Hq, Lq, dtype=torch.float32, device=q.device)
+    if counts is None:
+        counts = torch.empty(B, Hq, dtype=torch.int32, device=q.device)
+    nbytes = ssa_decode_workspace_bytes(B, Hq, Lq, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    st = ssa_decode(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale, lam, Bc,
+                    num_splits, workspace, workspace.numel() * workspace.element_size(), stream)
+    if st != SSA_OK:
+        raise SSAError(st, "ssa_decode")
     return out, lse, counts

@@ -29,7 +29,8 @@ def _declared_functions():
 def test_header_declares_the_entry_points():
     assert _declared_functions() == sorted(
         ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
-         "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version"])
+         "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version",
+         "ssa_decode", "ssa_decode_workspace_bytes"])
 
 
 def test_library_exports_every_declared_symbol(ssa):
@@ -104,3 +105,35 @@ def test_visited_tiles_closed_forms(ssa):
     assert ssa.ssa_visited_tiles(0, 75600, 75600, 128, 128) == 591 * 591
     assert ssa.ssa_visited_tiles(1, 256, 256, 64, 64) == 10
     assert ssa.ssa_visited_tiles(1, 0, 5, 64, 64) == -1
+
+
+def _dcall(ssa, **over):
+    a = dict(q=0x1000, k=0x2000, v=0x3000, out=0x4000, lse=0x5000, cnt=0x6000, B=2, Hq=8, Hkv=2,
+             Lq=1, Lk=4096, d=128, causal=1, scale=0.088, lam=1e-4, Bc=128, splits=4, ws=0x7000,
+             wsb=None)
+    a.update(over)
+    wsb = a["wsb"] if a["wsb"] is not None else ssa.ssa_decode_workspace_bytes(a["B"], a["Hq"], a["Lq"], a["d"],
+                                                                               max(a["splits"], 1))
+    return ssa.lib.ssa_decode(a["q"], a["k"], a["v"], a["out"], a["lse"], a["cnt"], a["B"], a["Hq"],
+                              a["Hkv"], a["Lq"], a["Lk"], a["d"], a["causal"], a["scale"], a["lam"],
+                              a["Bc"], a["splits"], a["ws"], wsb, None)
+
+
+@pytest.mark.parametrize("over", [
+    dict(q=0), dict(v=0), dict(ws=0), dict(cnt=0), dict(B=0), dict(Lk=0), dict(splits=0),
+    dict(Hq=6, Hkv=4), dict(scale=0.0), dict(lam=-1.0), dict(lam=float("nan")), dict(k=0x2004),
+    dict(wsb=16),
+])
+def test_decode_invalid_arguments(ssa, over):
+    assert _dcall(ssa, **over) == ssa.SSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("over", [dict(d=96), dict(Bc=32), dict(Lq=9), dict(Hq=64, Hkv=1)])
+def test_decode_unsupported_arguments(ssa, over):
+    assert _dcall(ssa, **over) == ssa.SSA_ERR_UNSUPPORTED
+
+
+def test_decode_workspace_bytes(ssa):
+    # partial accumulators (fp32 d per row and split), (max, sum) per row and split, skip counts
+    assert ssa.ssa_decode_workspace_bytes(8, 32, 1, 128, 16) == 8 * 32 * 16 * (128 * 4 + 8) + 8 * 32 * 16 * 4
+    assert ssa.ssa_decode_workspace_bytes(0, 32, 1, 128, 16) == 0

@@ -1,0 +1,108 @@
+"""GPU parity of the split-KV decode path (ssa_decode through the C ABI)
+against the fp64 decode oracle (oracle/decode.py), on the same seeded bf16
+inputs: outputs max-abs <= 2e-2 and relative L2 <= 5e-3, lse max-abs <= 1e-3,
+per-head skip counts equal except tiles whose decision margin is within
+1e-3 * lambda (the oracle marks them)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle.decode import decode as decode_oracle
+from softmax_ssa_fwd_b200.inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+OUT_MAX_ABS, OUT_REL_L2, LSE_MAX_ABS = 2e-2, 5e-3, 1e-3
+
+
+def _gen(B, Hq, Hkv, Lq, Lk, d, seed, sink_coef):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, Lq, Hq, d, generator=g)
+    k = torch.randn(B, Lk, Hkv, d, generator=g)
+    v = torch.randn(B, Lk, Hkv, d, generator=g)
+    if sink_coef:
+        u = torch.randn(d, generator=g)
+        u /= u.norm()
+        q += sink_coef * u
+        k[:, :4] += sink_coef * u
+    return q.bfloat16(), k.bfloat16(), v.bfloat16()
+
+
+def _check(q, k, v, *, causal, scale, lam, Bc, splits, heads=None):
+    from softmax_ssa_fwd_b200 import ssa
+    out, lse, cnt = ssa.decode(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale, lam=lam,
+                               Bc=Bc, num_splits=splits)
+    torch.cuda.synchronize()
+    ref = decode_oracle(q, k, v, causal=causal, scale=scale, lam=lam, Bc=Bc, num_splits=splits,
+                        heads=heads)
+    o = out.float().cpu().numpy()
+    ls = lse.cpu().numpy()
+    c = cnt.cpu().numpy()
+    B, Lq, Hq, d = q.shape
+    pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    num = den = 0.0
+    worst = 0.0
+    for b, h in pairs:
+        diff = o[b, :, h] - ref.out[b, :, h]
+        worst = max(worst, float(np.abs(diff).max()))
+        num += float((diff ** 2).sum())
+        den += float((ref.out[b, :, h] ** 2).sum())
+        fin = np.isfinite(ref.lse[b, h])
+        assert np.array_equal(fin, np.isfinite(ls[b, h])), (b, h)
+        if fin.any():
+            assert np.abs(ls[b, h][fin] - ref.lse[b, h][fin]).max() <= LSE_MAX_ABS, (b, h)
+        margin = int(ref.marginal[b, h].sum())
+        assert abs(int(c[b, h]) - int(ref.skip_count[b, h])) <= margin, (b, h, c[b, h], ref.skip_count[b, h])
+    assert worst <= OUT_MAX_ABS, worst
+    assert (num / max(den, 1e-30)) ** 0.5 <= OUT_REL_L2
+    return ref, c
+
+
+CASES = [
+    # B, Hq, Hkv, Lq, Lk, d, causal, Bc, splits, lam, sink_coef
+    (2, 8, 2, 1, 1000, 128, True, 128, 1, 1e-3, 12.0),   # one split = the prefill rule; ragged tail
+    (2, 8, 2, 1, 1000, 128, True, 128, 4, 1e-3, 12.0),
+    (1, 8, 2, 3, 777, 64, True, 64, 5, 1e-2, 12.0),      # several query rows, causal inside the tile
+    (1, 4, 4, 2, 512, 128, False, 64, 3, 0.0, 3.0),      # lambda = 0: dense, MHA
+    (1, 16, 2, 4, 300, 64, True, 128, 2, 1e-2, 12.0),    # G * Lq = 32, the maximum
+    (1, 8, 2, 2, 900, 128, True, 128, 3, 2.0, 12.0),     # lambda > 1
+    (1, 4, 2, 1, 200, 128, True, 128, 8, 1e-3, 12.0),    # more splits than key tiles
+    (1, 32, 8, 1, 4096, 128, True, 128, 16, 1e-4, 3.0),  # decode shape, literal inputs
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_decode_matches_oracle(case):
+    B, Hq, Hkv, Lq, Lk, d, causal, Bc, splits, lam, sc = case
+    q, k, v = _gen(B, Hq, Hkv, Lq, Lk, d, seed=hash(case) % 1000, sink_coef=sc)
+    ref, cnt = _check(q, k, v, causal=causal, scale=d ** -0.5, lam=lam, Bc=Bc, splits=splits)
+    nK = -(-Lk // Bc)
+    if sc >= 12.0 and 0 < lam <= 1e-2 and nK >= 2 * splits:
+        assert cnt.sum() > 0  # the skip path ran (a split's first tile is never skipped)
+
+
+def test_decode_one_split_equals_prefill_kernel():
+    """Same rule, two kernels: with one split the decode path must reproduce
+    the prefill kernel's skip counts exactly and its outputs within bf16."""
+    from softmax_ssa_fwd_b200 import ssa
+    q, k, v = _gen(1, 8, 2, 1, 1500, 128, seed=77, sink_coef=12.0)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    od, ld, cd = ssa.decode(qc, kc, vc, causal=True, scale=128 ** -0.5, lam=1e-3, Bc=128, num_splits=1)
+    of, lf, cf = ssa.attention(qc, kc, vc, causal=True, scale=128 ** -0.5, mode=ssa.MODE_SKIP, lam=1e-3,
+                               Br=128, Bc=128)
+    torch.cuda.synchronize()
+    assert torch.equal(cd.cpu(), cf[:, :, 0].cpu())
+    assert (od.float() - of.float()).abs().max().item() <= 2e-2
+    assert (ld - lf).abs().max().item() <= 1e-3
+
+
+def test_decode_workload_full_size_sampled_heads():
+    """The bench's decode workload at full size and its launch configuration,
+    checked on a sample of (sequence, head) pairs."""
+    w = WORKLOADS["qwen32k_decode"]
+    q, k, v = make_inputs(w, "cpu")
+    g = torch.Generator().manual_seed(9)
+    heads = sorted({(int(torch.randint(w.B, (1,), generator=g)), int(torch.randint(w.Hq, (1,), generator=g)))
+                    for _ in range(12)} | {(0, 0), (w.B - 1, w.Hq - 1)})
+    _check(q, k, v, causal=w.causal, scale=w.scale, lam=w.lambdas[0], Bc=w.Bc, splits=w.splits,
+           heads=heads)
