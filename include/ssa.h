@@ -119,6 +119,28 @@ int ssa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, floa
                     int causal, float scale, int mode, float lambda, int n, int m, int sink,
                     int recent, int Br, int Bc, void* stream);
 
+/* Forward pass over caller-selected key blocks.  The block-sparse page of the
+ * same stack ("Bitmask format": packed UInt32 exact-block bitmaps owned per
+ * (batch, KV head, Q block), one bit per KV block, padding bits in the final
+ * word ignored) gives the selection format; this entry consumes it on the
+ * skip-softmax path.  Everything else is ssa_fwd's: modes, layouts, outputs.
+ *   block_mask: [B, Hkv, nQ, ceil(nK / 32)] uint32, device, 4-byte aligned,
+ *               nQ = ceil(Lq / Br), nK = ceil(Lk / Bc); bit kt of word kt / 32
+ *               of (b, hkv, qt) selects key tile kt for query tile qt of every
+ *               query head that reads KV head hkv.  Bits of key tiles the query
+ *               tile cannot see (causal) and padding bits are ignored.
+ * A key tile whose bit is clear is not visited: no scores, no exponentials, no
+ * P.V, not counted in tile_skip_count; the skip-softmax recurrence (when
+ * SSA_MODE_SKIP is set) runs over the selected tiles in ascending order.  A
+ * query row with no selected visible key gets out = 0 and lse = -inf.
+ * Omitted blocks are dropped, not approximated (no proxy compensation).
+ * Limit: nK <= 2048 (SSA_ERR_UNSUPPORTED beyond).  Returns the status codes of
+ * ssa_fwd; SSA_ERR_INVALID_ARG for a NULL or misaligned block_mask. */
+int ssa_fwd_blockmask(const void* q, const void* k, const void* v, void* out, float* lse,
+                      int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                      int causal, float scale, int mode, float lambda, int n, int m, int sink,
+                      int recent, int Br, int Bc, const uint32_t* block_mask, void* stream);
+
 /* Total key tiles visited by all query tiles of one (batch, head) pair: a pure
  * function of the shape, used to turn skip counts into skip fractions and
  * executed FLOPs.  Returns -1 for invalid sizes. */

@@ -8,3 +8,5 @@ The arithmetic lives in ``ssa_oracle.c`` (plain C, fp64); this module only
 compiles it (``build()``) and marshals numpy arrays into it (``run_items``).
 """
 from .oracle import build, lib_path, run_items, visited_tiles, OracleResult  # noqa: F401
+# fp64 numpy oracles of the two further paths (same test-infrastructure rule):
+# oracle.decode (split-KV decode) and oracle.blockmask (caller-selected key blocks)

@@ -58,6 +58,8 @@ constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;  // default limit of a pipel
 // loads, MMAs) finish before it frees its memory; never shortened.
 constexpr uint64_t DRAIN_TIMEOUT_NS = 2000000000ull;
 constexpr float RESCALE_LOG2 = 8.0f;  // lazy O rescale once the max grew by 2^8
+// Key tiles a CTA can list when the caller selects key blocks by bitmap.
+constexpr int MAX_LISTED_TILES = 2048;
 // When POLY_EVERY > 0, one exp2 pair in POLY_EVERY runs as a polynomial on
 // the FMA pipe instead of the MUFU unit.  Measured on B200 (llama8k, wan) the
 // softmax here is latency-bound, not MUFU-bound, and every offload ratio
@@ -82,6 +84,7 @@ struct Params {
   float scale_log2;
   float log2_lambda;  // -inf for lambda == 0
   unsigned long long wait_ns;  // limit of each pipeline wait
+  const uint32_t* block_mask;  // optional [B, Hkv, nQ, nKw]: key blocks each query block visits
 };
 
 struct __align__(8) Bars {
@@ -94,6 +97,9 @@ struct __align__(8) Bars {
   uint32_t tmem_base;
   uint32_t vote[NQT][2];      // byte w: softmax warp w of the tile keeps the key tile
   uint32_t abort_flag;
+  int listed;                        // block-mask mode: key tiles in ktile[]
+  int listed_t[NQT];                 // of which tile t visits the first listed_t[t]
+  uint16_t ktile[MAX_LISTED_TILES];  // block-mask mode: the CTA's key tiles, ascending
 };
 
 template <int D, int BC>
@@ -320,9 +326,11 @@ struct Work {
   int nvis;               // per CTA
 };
 
-template <int D, int BC, int NM_M, bool DBG>
-__device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b, int hq, int t,
-                                             int pt, int nvis_h0, int nvis_h1, uint32_t tmem) {
+// VAR: 0 plain, 1 with debug outputs (skip / keep bits), 2 key blocks selected by bitmap.
+template <int D, int BC, int NM_M, int VAR>
+__device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b, int hq, int hkv,
+                                             int t, int pt, int nvis_h0, int nvis_h1, int nsteps,
+                                             uint32_t tmem) {
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int row = tid - 128 - 128 * t;
@@ -338,7 +346,9 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
   constexpr bool nm_on = NM_M != 0;
   const bool leader = p.half ? ((row & 63) == 0) : (row == 0);
   const int my_nvis = half ? nvis_h1 : nvis_h0;
-  const int nvis = nvis_h0 > nvis_h1 ? nvis_h0 : nvis_h1;
+  constexpr bool DBG = VAR == 1, MASK = VAR == 2;
+  const int nvis = nsteps;  // = max(nvis_h0, nvis_h1) unless key blocks are selected by bitmap
+  const bool vote_on = skip_on || MASK;
   // speculative exponentials are exact only while a skipped tile cannot raise the max
   const bool spec_ok = p.log2_lambda <= 0.f;
   bool prev_keep = true;
@@ -355,7 +365,23 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     bool ok = !failed && mbar_wait(smem_u32(&bars->s_full[t]), j & 1, p.wait_ns);
     ok = __all_sync(0xffffffffu, ok);
     float m_tile = -INFINITY;
-    const int col0 = j * BC;
+    // key tile of this step, and whether each logical query tile (half) of
+    // this tile visits it: visible, and selected when a bitmap is given
+    const int kt = MASK ? (int)bars->ktile[j] : j;
+    const int col0 = kt * BC;
+    auto visits = [&](int h) -> bool {
+      const int nv = h ? nvis_h1 : nvis_h0;
+      if constexpr (!MASK) {
+        return j < nv;
+      } else {
+        if (kt >= nv) return false;
+        const int qt = p.half ? 2 * pt + h : pt;
+        const uint32_t w = p.block_mask[((size_t)(b * p.Hkv + hkv) * p.nQ + qt) * p.nKw + (kt >> 5)];
+        return (w >> (kt & 31)) & 1u;
+      }
+    };
+    const bool vis0 = visits(0), vis1 = p.half ? visits(1) : vis0;
+    const bool my_vis = half ? vis1 : vis0;
     // Pass 1: the whole row of S in registers -- masks, N:M, tile row max.
     // The scores stay in registers through the vote and become P in pass 2.
     const bool need_mask = (col0 + BC > p.Lk) || (p.causal && col0 + BC - 1 > pos_first);
@@ -408,7 +434,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
         mx3 = fmax3(mx3, x[i + 6], x[i + 7]);
       }
       m_tile = fmaxf(fmax3(mx0, mx1, mx2), mx3);
-      if (DBG && p.keep_bits != nullptr && valid && j < my_nvis) {
+      if (DBG && p.keep_bits != nullptr && valid && my_vis) {
         uint32_t* kb = p.keep_bits + ((size_t)(b * p.Hq + hq) * p.Lq + grow) * p.Lkw;
 #pragma unroll
         for (int w = 0; w < BC / 32; ++w) {
@@ -435,14 +461,14 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     // the tile", and arrives on the tile's vote barrier for this step's
     // parity.  The MMA warp and the V producer read the same four bytes.
     const uint32_t vbar = smem_u32(&bars->vote_bar[t][j & 1]);
-    if (skip_on) {
-      const bool wkeep = !__all_sync(0xffffffffu, negligible) && j < my_nvis;
+    if (vote_on) {
+      const bool wkeep = (skip_on ? !__all_sync(0xffffffffu, negligible) : true) && my_vis;
       if (lane == 0) {
         st_shared_u8(smem_u32(&bars->vote[t][j & 1]) + quarter, wkeep ? 1u : 0u);
         mbar_arrive(vbar);
       }
     }
-    bool keep_h[2] = {j < nvis_h0, j < nvis_h1};
+    bool keep_h[2] = {vis0, vis1};
     // (warp-uniform outcome: the tcgen05 accesses that follow are warp-collective)
     auto decide = [&]() {
       if (!__all_sync(0xffffffffu, mbar_wait(vbar, (j >> 1) & 1, p.wait_ns))) {
@@ -459,7 +485,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     // nothing: the exponentials may start before the vote completes.  A
     // tile right after a skipped one waits for the vote instead, so long
     // runs of skipped tiles spend no MUFU time.
-    bool decided = !skip_on;
+    bool decided = !vote_on;
     if (!decided && !(spec_ok && prev_keep)) {
       decide();
       decided = true;
@@ -544,7 +570,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     const bool tile_keep = keep_h[0] || keep_h[1];
     const bool my_keep = half ? keep_h[1] : keep_h[0];
     prev_keep = tile_keep;
-    if (leader && j < my_nvis) {
+    if (leader && my_vis) {
       if (!my_keep) {
         ++skipped;
         skip_word |= 1u << (j & 31);
@@ -608,7 +634,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
   }
 }
 
-template <int D, int BC, int NM_M, bool DBG>
+template <int D, int BC, int NM_M, int VAR>
 __global__ void __launch_bounds__(NTHREADS, 1)
     ssa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -623,6 +649,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool skip_on = (p.mode & SSA_MODE_SKIP) != 0;
+  // the MMA warp and the V producer read the softmax's per-step keep bytes
+  // whenever a tile may be left out: skip-softmax, or key blocks selected by bitmap
+  constexpr bool MASK = VAR == 2;
+  const bool vote_on = skip_on || MASK;
 
   // ---- work item: heaviest causal pairs first; query heads that share a KV
   // head are adjacent in launch order.
@@ -653,7 +683,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (wk.nvis_t[t] > wk.nvis) wk.nvis = wk.nvis_t[t];
     }
   }
-  const int nvis = wk.nvis;
+  int nvis = wk.nvis;
+
+  // ---- block-mask mode: the CTA walks the key tiles that any of its logical
+  // query tiles selects and can see, in ascending order (warp 3 lists them)
+  if (MASK && warp == 3) {
+    int last[4], qts[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int t = x >> 1, h = x & 1;
+      last[x] = wk.nvis_h[t][h] - 1;  // last visible key tile (-1: none)
+      qts[x] = p.half ? 2 * wk.pt[t] + h : wk.pt[t];
+    }
+    const int maxlast = max(max(last[0], last[1]), max(last[2], last[3]));
+    const int last_t0 = max(last[0], last[1]), last_t1 = max(last[2], last[3]);
+    int count = 0, c0 = 0, c1 = 0;
+    for (int base = 0; base <= maxlast; base += 32) {
+      const int kt = base + lane;
+      bool any = false;
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        if (kt <= last[x]) {
+          const uint32_t w = p.block_mask[((size_t)(wk.b * p.Hkv + wk.hkv) * p.nQ + qts[x]) * p.nKw + (kt >> 5)];
+          any |= ((w >> (kt & 31)) & 1u) != 0u;
+        }
+      }
+      const uint32_t bal = __ballot_sync(0xffffffffu, any);
+      const int pos = count + __popc(bal & ((1u << lane) - 1u));
+      if (any && pos < MAX_LISTED_TILES) bars->ktile[pos] = (uint16_t)kt;
+      count += __popc(bal);
+      c0 += __popc(__ballot_sync(0xffffffffu, any && kt <= last_t0));
+      c1 += __popc(__ballot_sync(0xffffffffu, any && kt <= last_t1));
+    }
+    if (lane == 0) {
+      bars->listed = min(count, MAX_LISTED_TILES);
+      bars->listed_t[0] = min(c0, MAX_LISTED_TILES);
+      bars->listed_t[1] = min(c1, MAX_LISTED_TILES);
+    }
+  }
 
   // ---- set-up
   if (tid == 0) {
@@ -689,6 +756,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  if (MASK) {
+    wk.nvis_t[0] = bars->listed_t[0];
+    wk.nvis_t[1] = bars->listed_t[1];
+    nvis = wk.nvis = bars->listed;
+  }
+  auto key_tile = [&](int j) { return MASK ? (int)bars->ktile[j] : j; };
 
   if (warp < 4) {
     reg_dealloc<104>();
@@ -718,7 +791,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive_expect_tx(fb, L::K_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(k_s + slot * L::K_BYTES + c * BC * 128, &tm_k, fb, c * 64, wk.hkv, j * BC, wk.b);
+          tma_load_4d(k_s + slot * L::K_BYTES + c * BC * 128, &tm_k, fb, c * 64, wk.hkv, key_tile(j) * BC, wk.b);
         issued = j + 1;
       }
       // drain: the newest load of each slot (older ones were consumed)
@@ -743,7 +816,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int t = 0; t < NQT; ++t) {
           if (j >= wk.nvis_t[t]) continue;
           bool keep = true;
-          if (skip_on) {
+          if (vote_on) {
             if (!mbar_wait_fast(smem_u32(&bars->vote_bar[t][j & 1]), (j >> 1) & 1, p.wait_ns)) {
               fail = true;
               break;
@@ -754,7 +827,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_arrive_expect_tx(fb, L::V_BYTES);
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
-              tma_load_4d(v_s + slot * L::V_BYTES + c * BC * 128, &tm_v, fb, c * 64, wk.hkv, j * BC, wk.b);
+              tma_load_4d(v_s + slot * L::V_BYTES + c * BC * 128, &tm_v, fb, c * 64, wk.hkv, key_tile(j) * BC, wk.b);
             last_load[slot] = j;
             loaded = true;
           }
@@ -818,7 +891,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int t = 0; t < NQT; ++t) {
           if (j >= wk.nvis_t[t]) continue;
           if (!mbar_wait_fast(smem_u32(&bars->p_ready[t]), j & 1, p.wait_ns)) { ok = false; break; }
-          const bool keep = !skip_on || ld_shared_u32(smem_u32(&bars->vote[t][j & 1])) != 0u;
+          const bool keep = !vote_on || ld_shared_u32(smem_u32(&bars->vote[t][j & 1])) != 0u;
           if (keep) {
             if (!v_seen) {
               if (!mbar_wait_fast(smem_u32(&bars->v_full[slot]), (j / VST) & 1, p.wait_ns)) { ok = false; break; }
@@ -862,9 +935,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     reg_alloc<200>();
     const int t = warp >> 3;  // warps 4-7: tile A, 8-11: tile B
-    softmax_tile<D, BC, NM_M, DBG>(p, bars, wk.b, wk.hq, t, t ? wk.pt[1] : wk.pt[0],
+    softmax_tile<D, BC, NM_M, VAR>(p, bars, wk.b, wk.hq, wk.hkv, t, t ? wk.pt[1] : wk.pt[0],
                                    t ? wk.nvis_h[1][0] : wk.nvis_h[0][0],
-                                   t ? wk.nvis_h[1][1] : wk.nvis_h[0][1], tmem);
+                                   t ? wk.nvis_h[1][1] : wk.nvis_h[0][1],
+                                   t ? wk.nvis_t[1] : wk.nvis_t[0], tmem);
   }
 
   // ---- teardown
@@ -888,7 +962,7 @@ static unsigned long long g_wait_ns = WAIT_TIMEOUT_NS;
 static EncodeTiledFn g_encode = nullptr;
 constexpr int MAX_DEV = 64;
 static int* g_status[MAX_DEV] = {};
-static bool g_attr_set[MAX_DEV][24] = {};
+static bool g_attr_set[MAX_DEV][36] = {};
 
 static EncodeTiledFn encode_fn() {
   if (g_encode) return g_encode;
@@ -927,36 +1001,40 @@ static int* status_word(int dev) {
   return g_status[dev];
 }
 
-template <int D, int BC, int NM_M, bool DBG>
+template <int D, int BC, int NM_M, int VAR>
 static int launch_one(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const Params& p, int grid, cudaStream_t stream, int dev, int inst) {
   using L = Smem<D, BC>;
   if (!g_attr_set[dev][inst]) {
-    if (cudaFuncSetAttribute(ssa_fwd_kernel<D, BC, NM_M, DBG>,
+    if (cudaFuncSetAttribute(ssa_fwd_kernel<D, BC, NM_M, VAR>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC) != cudaSuccess)
       return SSA_ERR_CUDA;
     g_attr_set[dev][inst] = true;
   }
-  ssa_fwd_kernel<D, BC, NM_M, DBG><<<grid, NTHREADS, L::ALLOC, stream>>>(mq, mk, mv, p);
+  ssa_fwd_kernel<D, BC, NM_M, VAR><<<grid, NTHREADS, L::ALLOC, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
 }
 
-// One instance per (N:M group width or none) x (debug outputs or not), so the
-// plain skip-softmax kernel carries no N:M or debug code.
+// One instance per (N:M group width or none) x (plain, debug outputs, key
+// blocks by bitmap), so the plain skip-softmax kernel carries no N:M, debug or
+// bitmap code.
+template <int D, int BC, int NM_M>
+static int launch_var(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const Params& p, int grid, cudaStream_t stream, int dev, int inst) {
+  if (p.block_mask != nullptr) return launch_one<D, BC, NM_M, 2>(mq, mk, mv, p, grid, stream, dev, inst + 2);
+  if (p.skip_bits != nullptr || p.keep_bits != nullptr)
+    return launch_one<D, BC, NM_M, 1>(mq, mk, mv, p, grid, stream, dev, inst + 1);
+  return launch_one<D, BC, NM_M, 0>(mq, mk, mv, p, grid, stream, dev, inst);
+}
+
 template <int D, int BC>
 static int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                   const Params& p, int grid, cudaStream_t stream, int dev, int base) {
-  const bool dbg = p.skip_bits != nullptr || p.keep_bits != nullptr;
   const int nm = (p.mode & SSA_MODE_NM) ? p.m : 0;
-  const int inst = base * 6 + (nm == 0 ? 0 : nm == 4 ? 2 : 4) + (dbg ? 1 : 0);
-  if (nm == 0)
-    return dbg ? launch_one<D, BC, 0, true>(mq, mk, mv, p, grid, stream, dev, inst)
-               : launch_one<D, BC, 0, false>(mq, mk, mv, p, grid, stream, dev, inst);
-  if (nm == 4)
-    return dbg ? launch_one<D, BC, 4, true>(mq, mk, mv, p, grid, stream, dev, inst)
-               : launch_one<D, BC, 4, false>(mq, mk, mv, p, grid, stream, dev, inst);
-  return dbg ? launch_one<D, BC, 8, true>(mq, mk, mv, p, grid, stream, dev, inst)
-             : launch_one<D, BC, 8, false>(mq, mk, mv, p, grid, stream, dev, inst);
+  const int inst = base * 9 + (nm == 0 ? 0 : nm == 4 ? 3 : 6);
+  if (nm == 0) return launch_var<D, BC, 0>(mq, mk, mv, p, grid, stream, dev, inst);
+  if (nm == 4) return launch_var<D, BC, 4>(mq, mk, mv, p, grid, stream, dev, inst);
+  return launch_var<D, BC, 8>(mq, mk, mv, p, grid, stream, dev, inst);
 }
 
 static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -965,7 +1043,7 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
                int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
                float scale, int mode, float lambda, int n, int m, int sink, int recent, int Br,
                int Bc, void* stream, uint32_t* skip_bits, uint32_t* keep_bits,
-               int* status_override = nullptr) {
+               int* status_override = nullptr, const uint32_t* block_mask = nullptr) {
   // ---- argument checks (synchronous, nothing launched on failure)
   if (!q || !k || !v || !out || !lse || !tile_skip_count) return SSA_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Lk <= 0 || d <= 0) return SSA_ERR_INVALID_ARG;
@@ -981,6 +1059,10 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
   if (mode & SSA_MODE_NM) {
     if (!((m == 4 && n >= 1 && n <= 4) || (m == 8 && n >= 1 && n <= 8))) return SSA_ERR_UNSUPPORTED;
     if (Bc % m != 0) return SSA_ERR_UNSUPPORTED;
+  }
+  if (block_mask != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(block_mask) & 3u) != 0u) return SSA_ERR_INVALID_ARG;
+    if ((Lk + Bc - 1) / Bc > MAX_LISTED_TILES) return SSA_ERR_UNSUPPORTED;
   }
   const long long nQp = (Lq + BM - 1) / BM;
   const long long grid = ((nQp + 1) / 2) * B * Hq;
@@ -1022,6 +1104,7 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
   p.log2_lambda = ((mode & SSA_MODE_SKIP) && lambda > 0.f) ? (float)std::log2((double)lambda)
                                                            : -INFINITY;
   p.wait_ns = g_wait_ns;
+  p.block_mask = block_mask;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // A caller-supplied status word (the allocation-free entry point's shared
   // scratch) keeps the previous call's contents: clear it on the stream first.
@@ -1105,6 +1188,15 @@ int ssa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, floa
                     int recent, int Br, int Bc, void* stream) {
   return ssa::run_noalloc(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale,
                           mode, lambda, n, m, sink, recent, Br, Bc, stream);
+}
+
+int ssa_fwd_blockmask(const void* q, const void* k, const void* v, void* out, float* lse,
+                      int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                      int causal, float scale, int mode, float lambda, int n, int m, int sink,
+                      int recent, int Br, int Bc, const uint32_t* block_mask, void* stream) {
+  if (!block_mask) return SSA_ERR_INVALID_ARG;
+  return ssa::run(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
+                  lambda, n, m, sink, recent, Br, Bc, stream, nullptr, nullptr, nullptr, block_mask);
 }
 
 int64_t ssa_visited_tiles(int causal, int Lq, int Lk, int Br, int Bc) {

@@ -25,7 +25,7 @@ MODE_DENSE, MODE_SKIP, MODE_NM = 0, 1, 2
 
 EXPORTED = ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
             "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version",
-            "ssa_decode", "ssa_decode_workspace_bytes"]
+            "ssa_decode", "ssa_decode_workspace_bytes", "ssa_fwd_blockmask"]
 
 
 class SSAError(RuntimeError):
@@ -56,6 +56,8 @@ def _load():
     lib.ssa_status_string.argtypes = [I]
     lib.ssa_version.restype = I
     lib.ssa_version.argtypes = []
+    lib.ssa_fwd_blockmask.restype = I
+    lib.ssa_fwd_blockmask.argtypes = fwd_args[:-1] + [P, P]
     lib.ssa_decode.restype = I
     lib.ssa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, F, I, I, P, ctypes.c_size_t, P]
     lib.ssa_decode_workspace_bytes.restype = ctypes.c_size_t
@@ -199,4 +201,32 @@ def decode(q, k, v, *, causal=True, scale=None, lam=0.0, Bc=128, num_splits=None
                     num_splits, workspace, workspace.numel() * workspace.element_size(), stream)
     if st != SSA_OK:
         raise SSAError(st, "ssa_decode")
+    return out, lse, counts
+
+
+def ssa_fwd_blockmask(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
+                      lam, n, m, sink, recent, Br, Bc, block_mask, stream=None) -> int:
+    """The key-block-selecting entry point (see include/ssa.h); returns its status code."""
+    return lib.ssa_fwd_blockmask(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                 _ptr(tile_skip_count), B, Hq, Hkv, Lq, Lk, d, int(causal),
+                                 float(scale), int(mode), float(lam), int(n), int(m), int(sink),
+                                 int(recent), Br, Bc, _ptr(block_mask), _stream(stream))
+
+
+def attention_blockmask(q, k, v, block_mask, *, causal=True, scale=None, mode=MODE_SKIP, lam=0.0,
+                        n=0, m=0, sink=0, recent=0, Br=128, Bc=128, stream=None):
+    """Forward over the key blocks selected by ``block_mask`` ([B, Hkv, nQ, ceil(nK/32)]
+    int32/uint32 CUDA tensor).  Returns (out, lse, tile_skip_count) like ``attention``."""
+    B, Lq, Hq, d = q.shape
+    _, Lk, Hkv, _ = k.shape
+    if scale is None:
+        scale = d ** -0.5
+    nQ = -(-Lq // Br)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, Lq, dtype=torch.float32, device=q.device)
+    counts = torch.empty(B, Hq, nQ, dtype=torch.int32, device=q.device)
+    st = ssa_fwd_blockmask(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode, lam,
+                           n, m, sink, recent, Br, Bc, block_mask, stream)
+    if st != SSA_OK:
+        raise SSAError(st, "ssa_fwd_blockmask")
     return out, lse, counts

@@ -30,7 +30,7 @@ def test_header_declares_the_entry_points():
     assert _declared_functions() == sorted(
         ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
          "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version",
-         "ssa_decode", "ssa_decode_workspace_bytes"])
+         "ssa_decode", "ssa_decode_workspace_bytes", "ssa_fwd_blockmask"])
 
 
 def test_library_exports_every_declared_symbol(ssa):
@@ -137,3 +137,12 @@ def test_decode_workspace_bytes(ssa):
     # partial accumulators (fp32 d per row and split), (max, sum) per row and split, skip counts
     assert ssa.ssa_decode_workspace_bytes(8, 32, 1, 128, 16) == 8 * 32 * 16 * (128 * 4 + 8) + 8 * 32 * 16 * 4
     assert ssa.ssa_decode_workspace_bytes(0, 32, 1, 128, 16) == 0
+
+
+def test_blockmask_argument_checks(ssa):
+    base = (0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 1, 4, 2, 256, 256, 128, 1, 0.088, 1,
+            1e-3, 2, 4, 4, 128, 128, 128)
+    assert ssa.lib.ssa_fwd_blockmask(*base, None, None) == ssa.SSA_ERR_INVALID_ARG      # no mask
+    assert ssa.lib.ssa_fwd_blockmask(*base, 0x7002, None) == ssa.SSA_ERR_INVALID_ARG    # misaligned
+    long = base[:10] + (2049 * 128,) + base[11:]
+    assert ssa.lib.ssa_fwd_blockmask(*long, 0x7000, None) == ssa.SSA_ERR_UNSUPPORTED   # > 2048 key tiles
