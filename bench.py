@@ -218,6 +218,33 @@ def run_reference(args, w, lam, rank, world):
     return 0
 
 
+def block_mask_bits(w, density: float, seed: int) -> np.ndarray:
+    """Seeded random key-block selection [B, Hkv, nQ, nK] (bool) restricted to the
+    visible tiles; key tile 0 and each query block's last visible tile are always
+    selected."""
+    nQ, nK = -(-w.L // w.Br), -(-w.L // w.Bc)
+    rng = np.random.default_rng(seed)
+    bits = rng.random((w.B, w.Hkv, nQ, nK)) < density
+    for qt in range(nQ):
+        last = min(nK - 1, (min(w.L, qt * w.Br + w.Br) - 1) // w.Bc) if w.causal else nK - 1
+        bits[:, :, qt, last + 1:] = False
+        bits[:, :, qt, 0] = True
+        bits[:, :, qt, last] = True
+    return bits
+
+
+def pack_bits(bits: np.ndarray) -> np.ndarray:
+    """[..., nK] bool -> [..., ceil(nK / 32)] uint32, bit kt % 32 of word kt // 32."""
+    nK = bits.shape[-1]
+    nKw = -(-nK // 32)
+    padded = np.zeros(bits.shape[:-1] + (nKw * 32,), dtype=np.uint32)
+    padded[..., :nK] = bits
+    words = np.zeros(bits.shape[:-1] + (nKw,), dtype=np.uint32)
+    for i in range(32):
+        words |= padded[..., i::32] << np.uint32(i)
+    return words
+
+
 def decode_cpu_baseline(w, lam, budget_s: float, seed: int = 7):
     """The fp64 decode oracle (numpy) on a bounded sample of (sequence, head)
     pairs of the decode workload; dense-equivalent FLOPs of the sample / wall."""
@@ -370,6 +397,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--mask-density", type=float, default=0.0,
+                    help="select key blocks by a seeded random bitmap of this density "
+                         "(ssa_fwd_blockmask); key tile 0 and the diagonal tile always selected")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -414,11 +444,22 @@ def main():
         cnt = torch.empty(w.B, w.Hq, -(-w.L // w.Br), dtype=torch.int32, device=dev)
         sets.append((q, k, v, out, lse, cnt))
     stream = torch.cuda.current_stream(dev)
+    nQ, nK = -(-w.L // w.Br), -(-w.L // w.Bc)
+    mask_bits = mask_dev = None
+    if args.mask_density > 0:
+        mask_bits = block_mask_bits(w, args.mask_density, seed=w.seed + 31 * rank)
+        mask_dev = torch.from_numpy(pack_bits(mask_bits).view(np.int32)).to(dev)
+
+    def fwd(q, k, v, out, lse, cnt):
+        if mask_dev is not None:
+            return ssa.ssa_fwd_blockmask(q, k, v, out, lse, cnt, w.B, w.Hq, w.Hkv, w.L, w.L, w.d, w.causal,
+                                         w.scale, w.mode, lam, w.n, w.m, w.sink, w.recent, w.Br, w.Bc,
+                                         mask_dev, stream)
+        return ssa.ssa_fwd(q, k, v, out, lse, cnt, w.B, w.Hq, w.Hkv, w.L, w.L, w.d, w.causal, w.scale,
+                           w.mode, lam, w.n, w.m, w.sink, w.recent, w.Br, w.Bc, stream)
 
     def step(i):
-        q, k, v, out, lse, cnt = sets[i & 1]
-        st = ssa.ssa_fwd(q, k, v, out, lse, cnt, w.B, w.Hq, w.Hkv, w.L, w.L, w.d, w.causal, w.scale,
-                         w.mode, lam, w.n, w.m, w.sink, w.recent, w.Br, w.Bc, stream)
+        st = fwd(*sets[i & 1])
         if st != 0:
             raise RuntimeError(ssa.status_string(st))
 
@@ -451,6 +492,8 @@ def main():
 
     # skip statistics of the timed workload (identical every step per input set)
     visited = ssa.ssa_visited_tiles(w.causal, w.L, w.L, w.Br, w.Bc) * w.B * w.Hq
+    if mask_bits is not None:  # selected visible tiles, per KV head times its query heads
+        visited = int(mask_bits.sum()) * (w.Hq // w.Hkv)
     skipped = sum(int(s[5].sum()) for s in sets) / len(sets)
     kept = visited - skipped
     flops_dense = dense_equiv_flops(w)
@@ -483,8 +526,7 @@ def main():
             dq.copy_(hq_, non_blocking=True)
             dk.copy_(hk_, non_blocking=True)
             dv.copy_(hv_, non_blocking=True)
-            st = ssa.ssa_fwd(dq, dk, dv, out, lse, cnt, w.B, w.Hq, w.Hkv, w.L, w.L, w.d, w.causal,
-                             w.scale, w.mode, lam, w.n, w.m, w.sink, w.recent, w.Br, w.Bc, stream)
+            st = fwd(dq, dk, dv, out, lse, cnt)
             if st != 0:
                 raise RuntimeError(ssa.status_string(st))
             ho.copy_(out, non_blocking=True)
@@ -517,7 +559,9 @@ def main():
             "value": tflops_dense, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload_name(w, lam), "parallelism": f"replicas x{world}",
+            "config": {"workload": workload_name(w, lam) + (f" key blocks by bitmap, density "
+                                                             f"{args.mask_density:g}" if mask_bits is not None else ""),
+                       "parallelism": f"replicas x{world}",
                        "l2": "inputs alternate between 2 sets of 168 MB each (> 126 MB L2)"},
             "executed_tflops": tflops_exec,
             "executed_frac_of_peak": tflops_exec / world / bf16_peak,

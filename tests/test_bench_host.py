@@ -62,3 +62,20 @@ def test_two_gloo_ranks_take_the_max_time():
 def test_single_process_identity():
     assert bench.reduce_max(3.5, None, torch.device("cpu")) == 3.5
     assert bench.job_rate(10.0, 1, 2.0) == pytest.approx(5000.0)
+
+
+def test_block_mask_helpers():
+    import numpy as np
+    import bench
+    from oracle.blockmask import block_selected
+    from softmax_ssa_fwd_b200.inputs import WORKLOADS
+    w = WORKLOADS["llama8k"].with_(L=1000, Hq=4, Hkv=2)
+    bits = bench.block_mask_bits(w, 0.3, seed=3)
+    words = bench.pack_bits(bits)
+    nQ, nK = bits.shape[2], bits.shape[3]
+    for qt in range(nQ):
+        last = min(nK - 1, (min(w.L, qt * w.Br + w.Br) - 1) // w.Bc)
+        assert bits[:, :, qt, 0].all() and bits[:, :, qt, last].all()
+        assert not bits[:, :, qt, last + 1:].any()
+        for kt in range(nK):
+            assert block_selected(words, 0, 1, qt, kt) == bits[0, 1, qt, kt]
