@@ -397,6 +397,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--splits", type=int, default=None, help="decode: override the key splits")
     ap.add_argument("--mask-density", type=float, default=0.0,
                     help="select key blocks by a seeded random bitmap of this density "
                          "(ssa_fwd_blockmask); key tile 0 and the diagonal tile always selected")
@@ -409,6 +410,8 @@ def main():
         w = w.with_(sink_coef=args.sink_coef)
     if args.local_alpha is not None:
         w = w.with_(local_alpha=args.local_alpha)
+    if args.splits is not None:
+        w = w.with_(splits=args.splits)
     if args.L is not None:
         if w.rope == "3d":
             raise SystemExit("--L does not apply to the 3D-rotary video workload")

@@ -61,7 +61,7 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 template <int D, int BC, int RT>
-__global__ void __launch_bounds__(NT) decode_split_kernel(const Params p) {
+__global__ void __launch_bounds__(NT, RT <= 8 ? 2 : 1) decode_split_kernel(const Params p) {
   constexpr int TPK = NT / BC;       // threads per key in the score phase
   constexpr int DP = D / TPK;        // d slice per thread
   constexpr int NDP = D / 2;         // column pairs
@@ -126,8 +126,26 @@ __global__ void __launch_bounds__(NT) decode_split_kernel(const Params p) {
   };
   load_k(kt0);
 
+  // V pairs of the current tile; issued before the tile's scores when the
+  // previous tile was kept (so their latency hides behind the softmax), else
+  // only once the vote has kept this tile
+  constexpr int NV = BC / NKG;
+  uint32_t vraw[NV];
+  auto load_v = [&](int j0) {
+    const int ncols = min(BC, p.Lk - j0);
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+      const int c = kg + NKG * u;
+      vraw[u] = c < ncols ? *reinterpret_cast<const uint32_t*>(vbase + (size_t)(j0 + c) * kv_row + 2 * dpair)
+                          : 0u;
+    }
+  };
+  bool prev_any_keep = true;
+
   for (int kt = kt0; kt < kt1; ++kt) {
     const int j0 = kt * BC;
+    const bool v_early = prev_any_keep;
+    if (v_early) load_v(j0);
     // ---- scores: ss[r][c] = q_r . k_{j0+c} in log2 units (-inf where masked)
     {
       const int c = kc, part = kpart;
@@ -158,6 +176,8 @@ __global__ void __launch_bounds__(NT) decode_split_kernel(const Params p) {
         }
       }
     }
+    // the next tile's K is on its way during the rest of this tile
+    load_k(kt + 1);
     __syncthreads();
     // ---- tile row max and "negligible" per row
 #pragma unroll
@@ -225,27 +245,19 @@ __global__ void __launch_bounds__(NT) decode_split_kernel(const Params p) {
       }
     }
     __syncthreads();
-    // the next tile's K is on its way during this tile's P.V
-    load_k(kt + 1);
-    // ---- O += P V over the kept heads' rows; V is not read when no head keeps the tile
-    if (any_keep_s) {
+    // ---- O += P V over the kept heads' rows; V is not read when no head keeps the
+    // tile unless it was requested early (previous tile kept)
+    const bool any_keep = any_keep_s != 0;
+    prev_any_keep = any_keep;
+    if (any_keep) {
 #pragma unroll
       for (int r = 0; r < RT; ++r) {
         const float a = alpha_s[r];
         o0[r] *= a;
         o1[r] *= a;
       }
-      // all of this thread's V pairs of the tile first (independent loads), then the FMAs;
-      // columns past Lk read nothing and have P = 0
-      constexpr int NV = BC / NKG;
-      const int ncols = min(BC, p.Lk - j0);
-      uint32_t vraw[NV];
-#pragma unroll
-      for (int u = 0; u < NV; ++u) {
-        const int c = kg + NKG * u;
-        vraw[u] = c < ncols ? *reinterpret_cast<const uint32_t*>(vbase + (size_t)(j0 + c) * kv_row + 2 * dpair)
-                            : 0u;
-      }
+      // this thread's V pairs of the tile (columns past Lk read nothing and have P = 0)
+      if (!v_early) load_v(j0);
 #pragma unroll
       for (int u = 0; u < NV; ++u) {
         const int c = kg + NKG * u;
