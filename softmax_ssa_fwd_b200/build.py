@@ -6,7 +6,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = [os.path.join(HERE, "csrc", "ssa_fwd.cu"), os.path.join(HERE, "csrc", "ssa_decode.cu")]
-DEPS = SRC + [os.path.join(HERE, "csrc", "ptx.cuh"), os.path.join(ROOT, "include", "ssa.h")]
+DEPS = SRC + [os.path.join(HERE, "csrc", "ptx.cuh"), os.path.join(HERE, "csrc", "internal.h"),
+              os.path.join(ROOT, "include", "ssa.h")]
 LIB = os.path.join(HERE, "libssa.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

@@ -43,6 +43,7 @@
 #include <mutex>
 
 #include "../../include/ssa.h"
+#include "internal.h"
 #include "ptx.cuh"
 
 namespace ssa {
@@ -999,6 +1000,21 @@ static int* status_word(int dev) {
     g_status[dev] = w;
   }
   return g_status[dev];
+}
+
+bool tma_map_bf16(CUtensorMap* map, const void* base, int B, int L, int H, int d, int rows) {
+  std::lock_guard<std::mutex> g(g_mu);
+  return make_map(map, base, B, L, H, d, rows);
+}
+
+int* device_status_word(int dev) {
+  std::lock_guard<std::mutex> g(g_mu);
+  return status_word(dev);
+}
+
+unsigned long long wait_timeout_ns() {
+  std::lock_guard<std::mutex> g(g_mu);
+  return g_wait_ns;
 }
 
 template <int D, int BC, int NM_M, int VAR>
