@@ -8,29 +8,29 @@
 // tile when exp(tile_row_max - running_max) < lambda for every row.
 //
 // Decode reads the whole KV cache for a handful of query rows, so it is bound
-// by HBM; the arithmetic runs on the CUDA cores and each sequence's key tiles
-// are spread over `num_splits` CTAs per KV head.  Every split runs the
-// skip-softmax recurrence over its own key tiles in order, with its own
-// running max (its first tile is never skipped unless fully masked); a second
-// kernel merges the splits' (max, sum, accumulator) with the usual
-// log-sum-exp rule.  With one split this is exactly the prefill rule for a
-// single query tile.
+// by HBM; each sequence's key tiles are spread over `num_splits` CTAs per KV
+// head.  Every split runs the skip-softmax recurrence over its own key tiles
+// in order, with its own running max (its first tile is never skipped unless
+// fully masked); a second kernel merges the splits' (max, sum, accumulator)
+// with the usual log-sum-exp rule.  With one split this is exactly the
+// prefill rule for a single query tile.
 //
 // CTA (split s, KV head, batch): the G = Hq / Hkv query heads that share the
-// KV head, Lq rows each, R = G * Lq <= 32 rows in all; a key tile is decided
-// per query head (its Lq rows).  288 threads:
-//   warp 8     producer: TMA loads of each key tile's K and V (128-byte
-//              swizzled 64-column boxes) into an NS-stage shared-memory ring,
-//              running up to NS tiles ahead of the arithmetic.  Decode is
-//              bound by these bytes, so V is fetched with K: a skipped tile
-//              saves its exponentials and P.V, not its V bytes.
-//   warps 0-7  scores: thread t takes key t / TPK and a 1/TPK slice of d from
-//              shared memory, q.k against all R rows (packed fp32x2 FMAs),
-//              slices combined by shuffles; softmax: warp w owns rows w,
-//              w + 8, ...: tile row max, vote, P, row sum; P.V: each thread
-//              two output columns and every (256 / (d/2))-th key of the tile,
-//              partial accumulators of all R rows in registers, summed over
-//              threads through shared memory at the end of the split.
+// KV head, Lq rows each, R = G * Lq <= 32 rows in all, stacked as rows of one
+// 128-row query tile (the rest zero); a key tile is decided per query head
+// (its Lq rows).  160 threads:
+//   warp 0   producer: TMA loads of each key tile's K and V (128-byte swizzled
+//            64-column boxes) into an NS-stage shared-memory ring, up to NS
+//            tiles ahead.  Decode is bound by these bytes, so V is fetched
+//            with K: a skipped tile saves its exponentials and P.V, not its
+//            V bytes.
+//   warp 1   TMEM owner and MMA issuer: S = Q K^T into TMEM columns [0, Bc),
+//            O += P V into columns [128, 128 + d) with P read from TMEM, on
+//            tcgen05 (M = 128: the padding rows cost tensor time, which decode
+//            has to spare, and no CUDA-core arithmetic)
+//   warp 4   softmax: lane r = query row r = TMEM lane r: masks, tile row max,
+//            the per-head vote (ballots), P -> TMEM as bf16 pairs, O rescale
+//            when a row's max grows, and the split's (max, sum, accumulator)
 // Every wait is bounded; a wait that gives up raises the per-device status
 // word that ssa_device_status reads.
 #include <cuda.h>
@@ -52,11 +52,11 @@ using ssa::mbar_init;
 using ssa::mbar_wait;
 using ssa::smem_u32;
 
-constexpr int NTC = 256;         // arithmetic threads (warps 0-7)
-constexpr int NT = NTC + 32;     // plus the producer warp
-constexpr int RMAX = 32;
+constexpr int NT = 160;          // warps 0 producer, 1 MMA, 2-3 idle, 4 softmax
+constexpr int RMAX = 32;         // query rows per CTA: TMEM lanes 0-31, the softmax warp's
 constexpr int NS = 3;            // K/V ring depth (tiles)
-constexpr uint32_t COMPUTE_BAR = 1;  // named barrier of the 256 arithmetic threads
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t O_COL = 128;  // S at TMEM columns [0, Bc), O at [128, 128 + d)
 constexpr unsigned long long DRAIN_NS = 2000000000ull;
 
 struct Params {
@@ -80,47 +80,28 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__device__ __forceinline__ void compute_sync() {
-  asm volatile("bar.sync %0, %1;" ::"r"(COMPUTE_BAR), "r"(NTC) : "memory");
-}
 
 template <int D, int BC>
 struct DecSmem {
+  static constexpr uint32_t Q_BYTES = 128 * D * 2;         // the query tile, rows padded to 128
   static constexpr uint32_t TILE_BYTES = BC * D * 2;        // one K or V tile
   static constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;   // K then V
   static constexpr uint32_t RING_BYTES = NS * STAGE_BYTES;
+  static constexpr uint32_t TOTAL = 1024 + Q_BYTES + RING_BYTES;  // + alignment slack
 };
 
-// Byte offset of element (row, col) of a [D/64 boxes][rows][64] tile written by
-// TMA with 128-byte swizzle: 16-byte unit u of row r lands at u ^ (r & 7).
-template <int BC>
-__device__ __forceinline__ uint32_t sw128(int row, int col) {
-  const int box = col >> 6, inrow = (col & 63) * 2;
-  return (uint32_t)(box * BC * 128 + row * 128 + ((((inrow >> 4) ^ row) & 7) << 4) + (inrow & 15));
-}
-
-template <int D, int BC, int RT>
+template <int D, int BC>
 __global__ void __launch_bounds__(NT, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const Params p) {
-  constexpr int TPK = NTC / BC;      // threads per key in the score phase
-  constexpr int DP = D / TPK;        // d slice per thread
-  constexpr int QP = DP + 4;         // padded slice stride: slices of a row start in different banks
-  constexpr int QSTR = TPK * QP;     // q row stride in shared memory
-  constexpr int NDP = D / 2;         // column pairs
-  constexpr int NKG = NTC / NDP;     // key groups in the P.V phase
   using L = DecSmem<D, BC>;
   extern __shared__ uint8_t dsm_raw[];
-  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-  float* qs = reinterpret_cast<float*>(ring + L::RING_BYTES);  // RT * QSTR; reused for the O reduction
-  float* ss = qs + RT * QSTR;                                   // RT * BC scores, then P
-  __shared__ float alpha_s[RT];
-  __shared__ float mt_s[RT];
-  __shared__ int neg_s[RT];
-  __shared__ int keep_s[RMAX];  // per query head
-  __shared__ int any_keep_s;
+  uint8_t* q_tile = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = q_tile + L::Q_BYTES;
   __shared__ uint64_t full_bar[NS], empty_bar[NS];
-  __shared__ int failed_s;
+  __shared__ uint64_t s_full, p_ready, o_done, mma_done;
+  __shared__ uint32_t tmem_base;
+  __shared__ uint32_t keep_word;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int s = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
@@ -132,15 +113,39 @@ __global__ void __launch_bounds__(NT, 1)
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
       mbar_init(smem_u32(&full_bar[i]), 1);
-      mbar_init(smem_u32(&empty_bar[i]), 8);  // one arrival per arithmetic warp
+      mbar_init(smem_u32(&empty_bar[i]), 1);
     }
-    failed_s = 0;
+    mbar_init(smem_u32(&s_full), 1);
+    mbar_init(smem_u32(&p_ready), 1);
+    mbar_init(smem_u32(&o_done), 1);
+    mbar_init(smem_u32(&mma_done), 1);
     ssa::fence_mbar_init();
   }
+  if (warp == 1) {
+    ssa::tmem_alloc(smem_u32(&tmem_base), TMEM_COLS);
+    ssa::tmem_relinquish();
+  }
+  // the query tile: row r = g * Lq + i (head hkv * G + g, query row i), rows
+  // R..127 zero; K-major with 128-byte swizzle, as the MMA's A operand
+  for (int e = tid; e < 128 * (D / 8); e += NT) {
+    const int r = e / (D / 8), u = e % (D / 8);
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (r < R) {
+      const int g = r / Lq, i = r % Lq;
+      val = *reinterpret_cast<const uint4*>(p.q + (((size_t)b * Lq + i) * p.Hq + hkv * G + g) * D + 8 * u);
+    }
+    const int box = u >> 3, unit = u & 7;
+    *reinterpret_cast<uint4*>(q_tile + box * 128 * 128 + r * 128 + ((unit ^ (r & 7)) << 4)) = val;
+  }
+  ssa::fence_proxy_async_smem();  // generic writes of the tile, then tensor-core reads
+  ssa::tc_fence_before();
   __syncthreads();
+  ssa::tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const uint32_t q_s = smem_u32(q_tile), ring_s = smem_u32(ring);
 
-  if (warp == 8) {
-    // ======================= producer =======================
+  if (warp == 0) {
+    // ======================= producer: K and V tiles by TMA =======================
     if (lane == 0 && ntiles > 0) {
       ssa::tma_prefetch_desc(&tm_k);
       ssa::tma_prefetch_desc(&tm_v);
@@ -149,12 +154,11 @@ __global__ void __launch_bounds__(NT, 1)
         const int st = t % NS;
         if (!mbar_wait(smem_u32(&empty_bar[st]), ((t / NS) & 1) ^ 1, p.wait_ns)) {
           atomicOr(p.status, 1);
-          *reinterpret_cast<volatile int*>(&failed_s) = 1;
           break;
         }
         const uint32_t fb = smem_u32(&full_bar[st]);
         mbar_arrive_expect_tx(fb, L::STAGE_BYTES);
-        const uint32_t kd = smem_u32(ring + st * L::STAGE_BYTES), vd = kd + L::TILE_BYTES;
+        const uint32_t kd = ring_s + st * L::STAGE_BYTES, vd = kd + L::TILE_BYTES;
         const int j0 = (kt0 + t) * BC;
 #pragma unroll
         for (int box = 0; box < D / 64; ++box) {
@@ -163,214 +167,182 @@ __global__ void __launch_bounds__(NT, 1)
         }
         issued = t + 1;
       }
-      // drain: every load issued has landed before the CTA may exit
-      bool drained = true;
+      bool drained = true;  // every load issued has landed before the CTA may exit
       for (int t = max(0, issued - NS); t < issued; ++t)
         drained &= mbar_wait(smem_u32(&full_bar[t % NS]), (t / NS) & 1, DRAIN_NS);
       if (!drained) atomicOr(p.status, 1);
     }
-    return;
-  }
-
-  // ======================= arithmetic warps =======================
-  // q rows: r = g * Lq + i -> head hkv * G + g, query row i
-  for (int e = tid; e < RT * D; e += NTC) {
-    const int r = e / D, dd = e % D;
-    float val = 0.f;
-    if (r < R) {
-      const int g = r / Lq, i = r % Lq;
-      val = __bfloat162float(p.q[(((size_t)b * Lq + i) * p.Hq + hkv * G + g) * D + dd]) * p.c;
-    }
-    qs[r * QSTR + (dd / DP) * QP + dd % DP] = val;
-  }
-  // per-row state, owned by warp r % 8 (every lane holds a copy)
-  float m_run[RT / 8 > 0 ? RT / 8 : 1], l_run[RT / 8 > 0 ? RT / 8 : 1];
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    if (lane == 0 && ntiles > 0) {
+      constexpr uint32_t idesc_qk = ssa::idesc_bf16_f32(128, BC, false, false);
+      constexpr uint32_t idesc_pv = ssa::idesc_bf16_f32(128, D, false, true);
+      // S = Q K_t^T into TMEM columns [0, BC)
+      auto issue_s = [&](int t) -> bool {
+        const int st = t % NS;
+        if (!mbar_wait(smem_u32(&full_bar[st]), (t / NS) & 1, p.wait_ns)) return false;
+        ssa::tc_fence_after();
+        const uint32_t k_s = ring_s + st * L::STAGE_BYTES;
 #pragma unroll
-  for (int u = 0; u < (RT / 8 > 0 ? RT / 8 : 1); ++u) {
-    m_run[u] = -INFINITY;
-    l_run[u] = 0.f;
-  }
-  const int dpair = tid % NDP, kg = tid / NDP;
-  float o0[RT], o1[RT];
-#pragma unroll
-  for (int r = 0; r < RT; ++r) o0[r] = o1[r] = 0.f;
-  int skipped_tiles = 0;  // per head, kept by thread g (< G)
-  bool failed = false;
-  compute_sync();
-
-  const int kc = tid / TPK, kpart = tid % TPK;
-  for (int t = 0; t < ntiles; ++t) {
-    const int kt = kt0 + t;
-    const int j0 = kt * BC;
-    const int st = t % NS;
-    bool ok = !failed && mbar_wait(smem_u32(&full_bar[st]), (t / NS) & 1, p.wait_ns);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok && !failed) {
-      if (lane == 0) atomicOr(p.status, 1);
-      failed = true;
-    }
-    const uint8_t* ks = ring + st * L::STAGE_BYTES;
-    const uint8_t* vs = ks + L::TILE_BYTES;
-    // ---- scores: ss[r][c] = q_r . k_{j0+c} in log2 units (-inf where masked)
-    {
-      const int c = kc, part = kpart;
-      const int j = j0 + c;
-      float kv[DP];
-#pragma unroll
-      for (int u = 0; u < DP / 8; ++u) {
-        const uint4 w = *reinterpret_cast<const uint4*>(ks + sw128<BC>(c, part * DP + 8 * u));
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const __nv_bfloat162 pr = *reinterpret_cast<const __nv_bfloat162*>(&ww[h]);
-          kv[8 * u + 2 * h] = __low2float(pr);
-          kv[8 * u + 2 * h + 1] = __high2float(pr);
+        for (int k16 = 0; k16 < D / 16; ++k16) {
+          const uint32_t qoff = (k16 >> 2) * (128 * 128) + (k16 & 3) * 32;
+          const uint32_t koff = (k16 >> 2) * (BC * 128) + (k16 & 3) * 32;
+          ssa::mma_ss(tmem, ssa::smem_desc_sw128(q_s + qoff, 16, 1024),
+                      ssa::smem_desc_sw128(k_s + koff, 16, 1024), idesc_qk, k16 > 0 ? 1u : 0u);
         }
+        ssa::mma_commit(smem_u32(&s_full));
+        return true;
+      };
+      bool ok = issue_s(0);
+      int pv_count = 0;
+      for (int t = 0; ok && t < ntiles; ++t) {
+        const int st = t % NS;
+        if (!mbar_wait(smem_u32(&p_ready), t & 1, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        if (*reinterpret_cast<volatile uint32_t*>(&keep_word)) {
+          // O += P V: P (bf16 pairs over the S columns) from TMEM, V from the stage
+          ssa::tc_fence_after();
+          const uint32_t v_s = ring_s + st * L::STAGE_BYTES + L::TILE_BYTES;
+#pragma unroll
+          for (int k16 = 0; k16 < BC / 16; ++k16)
+            ssa::mma_ts(tmem + O_COL, tmem + k16 * 8, ssa::smem_desc_sw128(v_s + k16 * 16 * 128, BC * 128, 1024),
+                        idesc_pv, (pv_count > 0 || k16 > 0) ? 1u : 0u);
+          ++pv_count;
+        }
+        ssa::mma_commit(smem_u32(&empty_bar[st]));  // the stage is free once these MMAs are done
+        // (S_{t+1} overwrites P_t: it follows the P.V in issue order)
+        if (t + 1 < ntiles) ok = issue_s(t + 1);
       }
-#pragma unroll
-      for (int r = 0; r < RT; ++r) {
-        const float4* qr = reinterpret_cast<const float4*>(&qs[r * QSTR + part * QP]);
-        uint64_t a2 = ssa::f2_pack(0.f, 0.f);
-#pragma unroll
-        for (int e4 = 0; e4 < DP / 4; ++e4) {
-          const float4 qv = qr[e4];
-          a2 = ssa::ffma2(ssa::f2_pack(qv.x, qv.y), ssa::f2_pack(kv[4 * e4], kv[4 * e4 + 1]), a2);
-          a2 = ssa::ffma2(ssa::f2_pack(qv.z, qv.w), ssa::f2_pack(kv[4 * e4 + 2], kv[4 * e4 + 3]), a2);
-        }
-        float lo, hi;
-        ssa::f2_unpack(a2, lo, hi);
-        float acc = lo + hi;
-#pragma unroll
-        for (int o = 1; o < TPK; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (part == 0) {
-          bool vis = (r < R) && (j < p.Lk);
-          if (p.causal && r < R) vis = vis && (j <= r % Lq + p.Lk - Lq);
-          ss[r * BC + c] = vis ? acc : -INFINITY;
-        }
+      if (!ok) atomicOr(p.status, 1);
+      ssa::mma_commit(smem_u32(&o_done));
+      ssa::mma_commit(smem_u32(&mma_done));
+      if (!mbar_wait(smem_u32(&mma_done), 0, DRAIN_NS)) atomicOr(p.status, 1);
+    }
+  } else if (warp == 4) {
+    // ======================= softmax: lane r = query row r = TMEM lane r =======================
+    const int r = lane;
+    const bool valid = r < R;
+    const int g = valid ? r / Lq : 0, i = valid ? r % Lq : 0;
+    const int pos = i + p.Lk - Lq;
+    const uint32_t head_mask = ((Lq >= 32) ? 0xffffffffu : ((1u << Lq) - 1u)) << ((lane < G ? lane : 0) * Lq);
+    float m_true = -INFINITY, l = 0.f;  // log2 units of scale * q.k
+    int n_pv = 0, skipped = 0;
+    bool failed = false;
+    for (int t = 0; t < ntiles; ++t) {
+      bool ok = !failed && mbar_wait(smem_u32(&s_full), t & 1, p.wait_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok && !failed) {
+        if (lane == 0) atomicOr(p.status, 1);
+        failed = true;
       }
-    }
-    compute_sync();
-    // ---- tile row max and "negligible" per row
+      ssa::tc_fence_after();
+      float x[BC];
 #pragma unroll
-    for (int u = 0; u < (RT + 7) / 8; ++u) {
-      const int r = warp + 8 * u;
-      if (r < RT) {
-        float mx = -INFINITY;
+      for (int c = 0; c < BC / 32; ++c) ssa::tmem_ld32f(tmem + 32 * c, &x[32 * c]);
+      ssa::tmem_wait_ld();
+      const int j0 = (kt0 + t) * BC;
+      int lim = p.Lk - 1 - j0;  // last visible key of this row, relative to the tile
+      if (p.causal && pos - j0 < lim) lim = pos - j0;
+      if (!valid || !ok) lim = -1;
+      float mt = -INFINITY;
 #pragma unroll
-        for (int q4 = 0; q4 < BC / 32; ++q4) mx = fmaxf(mx, ss[r * BC + lane + 32 * q4]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float mr = m_run[u];
-        const bool neg = (r >= R) || mx == -INFINITY || (mr != -INFINITY && (mx - mr) < p.log2_lambda);
-        if (lane == 0) {
-          mt_s[r] = mx;
-          neg_s[r] = neg ? 1 : 0;
-        }
+      for (int c = 0; c < BC; ++c) {
+        x[c] = (c > lim) ? -INFINITY : x[c] * p.c;
+        mt = fmaxf(mt, x[c]);
       }
-    }
-    compute_sync();
-    // ---- the vote, one decision per query head
-    if (tid < G) {
-      int all_neg = 1;
-      for (int i = 0; i < Lq; ++i) all_neg &= neg_s[tid * Lq + i];
-      keep_s[tid] = !all_neg;
-      if (all_neg) ++skipped_tiles;
-    }
-    compute_sync();
-    if (tid == 0) {
-      int any = 0;
-      for (int g = 0; g < G; ++g) any |= keep_s[g];
-      any_keep_s = any;
-    }
-    // ---- P for the rows of kept heads
+      const bool neg = mt == -INFINITY || (m_true != -INFINITY && (mt - m_true) < p.log2_lambda);
+      const uint32_t negs = __ballot_sync(0xffffffffu, neg || !valid);
+      // lane g < G holds head g's decision; every row reads its own head's
+      const bool head_keeps = lane < G && (negs & head_mask) != head_mask;
+      const uint32_t keeps = __ballot_sync(0xffffffffu, head_keeps);
+      if (lane < G && !head_keeps) ++skipped;
+      const bool mine = valid && ((keeps >> g) & 1u);
+      if (keeps != 0u) {
+        const float m_new = fmaxf(m_true, mt);
+        const bool grow = mine && m_true != -INFINITY && m_new > m_true;
+        const float alpha = grow ? ex2(m_true - m_new) : 1.f;
+        const float mref = (m_new == -INFINITY) ? 0.f : m_new;
+        float sum = 0.f;
 #pragma unroll
-    for (int u = 0; u < (RT + 7) / 8; ++u) {
-      const int r = warp + 8 * u;
-      if (r < RT) {
-        const bool keep = r < R && keep_s[r / Lq];
-        float a = 1.f;
-        if (keep) {
-          const float mr = m_run[u];
-          const float mn = fmaxf(mr, mt_s[r]);
-          a = (mr == -INFINITY) ? 0.f : ex2(mr - mn);
-          const float mref = (mn == -INFINITY) ? 0.f : mn;
-          float sum = 0.f;
+        for (int h = 0; h < BC / 64; ++h) {
+          uint32_t pk[32];
 #pragma unroll
-          for (int q4 = 0; q4 < BC / 32; ++q4) {
-            const int c = lane + 32 * q4;
-            const float pv = ex2(ss[r * BC + c] - mref);
-            ss[r * BC + c] = pv;
-            sum += pv;
+          for (int c2 = 0; c2 < 32; ++c2) {
+            const float p0 = mine ? ex2(x[64 * h + 2 * c2] - mref) : 0.f;
+            const float p1 = mine ? ex2(x[64 * h + 2 * c2 + 1] - mref) : 0.f;
+            sum += p0 + p1;
+            __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            pk[c2] = *reinterpret_cast<uint32_t*>(&pb);
           }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-          l_run[u] = l_run[u] * a + sum;
-          m_run[u] = mn;
-        } else {
-          // a head that skips this tile (or a padding row) adds nothing
-#pragma unroll
-          for (int q4 = 0; q4 < BC / 32; ++q4) ss[r * BC + lane + 32 * q4] = 0.f;
+          ssa::tmem_st32(tmem + 32 * h, pk);
         }
-        if (lane == 0) alpha_s[r] = keep ? a : 1.f;
+        if (__any_sync(0xffffffffu, grow) && n_pv > 0) {
+          // every earlier P.V finished before S_t did: rescale O in place
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            ssa::tmem_ld32(tmem + O_COL + 32 * cc, o);
+            ssa::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            ssa::tmem_st32(tmem + O_COL + 32 * cc, o);
+          }
+        }
+        if (mine) {
+          l = l * alpha + sum;
+          m_true = m_new;
+        }
+        ++n_pv;
+      }
+      ssa::tmem_wait_st();
+      if (lane == 0) *reinterpret_cast<volatile uint32_t*>(&keep_word) = keeps != 0u ? 1u : 0u;
+      ssa::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&p_ready));
+    }
+    // ---- end of the split: the unnormalised accumulator and (max, sum) per row
+    bool okf = true;
+    if (ntiles > 0) okf = mbar_wait(smem_u32(&o_done), 0, p.wait_ns);
+    okf = __all_sync(0xffffffffu, okf) && !failed;
+    if (!okf && lane == 0) atomicOr(p.status, 1);
+    ssa::tc_fence_after();
+    const int hq = hkv * G + g;
+    float* orow = p.o_part + ((((size_t)b * p.Hq + hq) * Lq + i) * p.S + s) * D;
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      if (okf && n_pv > 0) {
+        ssa::tmem_ld32(tmem + O_COL + 32 * cc, o);
+        ssa::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = 0u;
+      }
+      if (valid) {
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4)
+          reinterpret_cast<float4*>(orow + 32 * cc)[e4] =
+              make_float4(__uint_as_float(o[4 * e4]), __uint_as_float(o[4 * e4 + 1]),
+                          __uint_as_float(o[4 * e4 + 2]), __uint_as_float(o[4 * e4 + 3]));
       }
     }
-    compute_sync();
-    // ---- O += P V over the kept heads' rows (nothing when no head keeps the tile)
-    if (any_keep_s) {
-#pragma unroll
-      for (int r = 0; r < RT; ++r) {
-        const float a = alpha_s[r];
-        o0[r] *= a;
-        o1[r] *= a;
-      }
-#pragma unroll 4
-      for (int c = kg; c < BC; c += NKG) {
-        const __nv_bfloat162 vv = *reinterpret_cast<const __nv_bfloat162*>(vs + sw128<BC>(c, 2 * dpair));
-        const float v0 = __low2float(vv), v1 = __high2float(vv);  // zeros past Lk (TMA fill), and P = 0 there
-#pragma unroll
-        for (int r = 0; r < RT; ++r) {
-          const float pr = ss[r * BC + c];
-          o0[r] = fmaf(pr, v0, o0[r]);
-          o1[r] = fmaf(pr, v1, o1[r]);
-        }
-      }
+    if (valid) {
+      float* ml = p.ml_part + ((((size_t)b * p.Hq + hq) * Lq + i) * p.S + s) * 2;
+      ml[0] = m_true;
+      ml[1] = (okf && n_pv > 0) ? l : 0.f;
     }
-    // the stage's K and V are no longer read: hand it back to the producer
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&empty_bar[st]));
-    compute_sync();
+    if (lane < G) p.sk_part[((size_t)b * p.Hq + hkv * G + lane) * p.S + s] = skipped;
   }
 
-  // ---- end of the split: sum the P.V partials over key groups, write out
-  float* ob = qs;  // RT * D floats (qs holds RT * QSTR >= RT * D)
-  for (int e = tid; e < RT * D; e += NTC) ob[e] = 0.f;
-  compute_sync();
-#pragma unroll
-  for (int r = 0; r < RT; ++r) {
-    if (r < R) {
-      atomicAdd(&ob[r * D + 2 * dpair], o0[r]);
-      atomicAdd(&ob[r * D + 2 * dpair + 1], o1[r]);
-    }
+  // ---- teardown
+  ssa::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ssa::tc_fence_after();
+    ssa::tmem_dealloc(tmem, TMEM_COLS);
   }
-  compute_sync();
-  for (int e = tid; e < R * D; e += NTC) {
-    const int r = e / D, dd = e % D;
-    const int g = r / Lq, i = r % Lq;
-    const int hq = hkv * G + g;
-    p.o_part[((((size_t)b * p.Hq + hq) * Lq + i) * p.S + s) * D + dd] = ob[e];
-  }
-#pragma unroll
-  for (int u = 0; u < (RT + 7) / 8; ++u) {
-    const int r = warp + 8 * u;
-    if (r < R && lane == 0) {
-      const int g = r / Lq, i = r % Lq;
-      const int hq = hkv * G + g;
-      float* ml = p.ml_part + ((((size_t)b * p.Hq + hq) * Lq + i) * p.S + s) * 2;
-      ml[0] = m_run[u];
-      ml[1] = l_run[u];
-    }
-  }
-  if (tid < G) p.sk_part[((size_t)b * p.Hq + hkv * G + tid) * p.S + s] = skipped_tiles;
 }
 
 // Merge the splits of one (batch, head, query row): block of d/2 threads.
@@ -408,31 +380,22 @@ __global__ void decode_combine_kernel(const Params p) {
   }
 }
 
-template <int D, int BC, int RT>
-static int launch_rt(const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, cudaStream_t st) {
+template <int D, int BC>
+static int launch_bc(const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, cudaStream_t st) {
   using L = DecSmem<D, BC>;
-  const size_t smem = 1024 + L::RING_BYTES + (size_t)RT * ((NTC / BC) * (D / (NTC / BC) + 4) + BC) * 4;
   static bool attr_set[64] = {};  // per instance and device, before the first launch there
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SSA_ERR_CUDA;
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(decode_split_kernel<D, BC, RT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(decode_split_kernel<D, BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)L::TOTAL) != cudaSuccess)
       return SSA_ERR_CUDA;
     attr_set[dev] = true;
   }
-  decode_split_kernel<D, BC, RT><<<dim3(p.S, p.Hkv, p.B), NT, smem, st>>>(mk, mv, p);
+  decode_split_kernel<D, BC><<<dim3(p.S, p.Hkv, p.B), NT, L::TOTAL, st>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return SSA_ERR_CUDA;
   decode_combine_kernel<D><<<dim3(p.Lq, p.Hq, p.B), D / 2, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
-}
-
-template <int D, int BC>
-static int launch_bc(const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, cudaStream_t st) {
-  if (p.R <= 4) return launch_rt<D, BC, 4>(mk, mv, p, st);
-  if (p.R <= 8) return launch_rt<D, BC, 8>(mk, mv, p, st);
-  if (p.R <= 16) return launch_rt<D, BC, 16>(mk, mv, p, st);
-  return launch_rt<D, BC, 32>(mk, mv, p, st);
 }
 
 static size_t workspace_bytes(int B, int Hq, int Lq, int d, int S) {
