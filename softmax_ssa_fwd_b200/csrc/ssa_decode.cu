@@ -55,8 +55,11 @@ using ssa::smem_u32;
 constexpr int NT = 160;          // warps 0 producer, 1 MMA, 2-3 idle, 4 softmax
 constexpr int RMAX = 32;         // query rows per CTA: TMEM lanes 0-31, the softmax warp's
 constexpr int NS = 3;            // K/V ring depth (tiles)
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t O_COL = 128;  // S at TMEM columns [0, Bc), O at [128, 128 + d)
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t O_COL = 128;  // O at TMEM columns [128, 128 + d)
+// S of key tile t (then its P) at columns [256 * (t & 1), 256 * (t & 1) + Bc):
+// S_{t+1} is computed while the softmax of tile t runs
+__device__ __forceinline__ uint32_t s_col(int t) { return 256u * (uint32_t)(t & 1); }
 constexpr unsigned long long DRAIN_NS = 2000000000ull;
 
 struct Params {
@@ -99,7 +102,7 @@ __global__ void __launch_bounds__(NT, 1)
   uint8_t* q_tile = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = q_tile + L::Q_BYTES;
   __shared__ uint64_t full_bar[NS], empty_bar[NS];
-  __shared__ uint64_t s_full, p_ready, o_done, mma_done;
+  __shared__ uint64_t s_full[2], p_ready, pv_done, o_done, mma_done;
   __shared__ uint32_t tmem_base;
   __shared__ uint32_t keep_word;
 
@@ -115,8 +118,10 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_init(smem_u32(&full_bar[i]), 1);
       mbar_init(smem_u32(&empty_bar[i]), 1);
     }
-    mbar_init(smem_u32(&s_full), 1);
+    mbar_init(smem_u32(&s_full[0]), 1);
+    mbar_init(smem_u32(&s_full[1]), 1);
     mbar_init(smem_u32(&p_ready), 1);
+    mbar_init(smem_u32(&pv_done), 1);
     mbar_init(smem_u32(&o_done), 1);
     mbar_init(smem_u32(&mma_done), 1);
     ssa::fence_mbar_init();
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (lane == 0 && ntiles > 0) {
       constexpr uint32_t idesc_qk = ssa::idesc_bf16_f32(128, BC, false, false);
       constexpr uint32_t idesc_pv = ssa::idesc_bf16_f32(128, D, false, true);
-      // S = Q K_t^T into TMEM columns [0, BC)
+      // S_t = Q K_t^T into TMEM columns [s_col(t), s_col(t) + BC)
       auto issue_s = [&](int t) -> bool {
         const int st = t % NS;
         if (!mbar_wait(smem_u32(&full_bar[st]), (t / NS) & 1, p.wait_ns)) return false;
@@ -187,13 +192,14 @@ __global__ void __launch_bounds__(NT, 1)
         for (int k16 = 0; k16 < D / 16; ++k16) {
           const uint32_t qoff = (k16 >> 2) * (128 * 128) + (k16 & 3) * 32;
           const uint32_t koff = (k16 >> 2) * (BC * 128) + (k16 & 3) * 32;
-          ssa::mma_ss(tmem, ssa::smem_desc_sw128(q_s + qoff, 16, 1024),
+          ssa::mma_ss(tmem + s_col(t), ssa::smem_desc_sw128(q_s + qoff, 16, 1024),
                       ssa::smem_desc_sw128(k_s + koff, 16, 1024), idesc_qk, k16 > 0 ? 1u : 0u);
         }
-        ssa::mma_commit(smem_u32(&s_full));
+        ssa::mma_commit(smem_u32(&s_full[t & 1]));
         return true;
       };
       bool ok = issue_s(0);
+      if (ok && ntiles > 1) ok = issue_s(1);
       int pv_count = 0;
       for (int t = 0; ok && t < ntiles; ++t) {
         const int st = t % NS;
@@ -207,13 +213,15 @@ __global__ void __launch_bounds__(NT, 1)
           const uint32_t v_s = ring_s + st * L::STAGE_BYTES + L::TILE_BYTES;
 #pragma unroll
           for (int k16 = 0; k16 < BC / 16; ++k16)
-            ssa::mma_ts(tmem + O_COL, tmem + k16 * 8, ssa::smem_desc_sw128(v_s + k16 * 16 * 128, BC * 128, 1024),
-                        idesc_pv, (pv_count > 0 || k16 > 0) ? 1u : 0u);
+            ssa::mma_ts(tmem + O_COL, tmem + s_col(t) + k16 * 8,
+                        ssa::smem_desc_sw128(v_s + k16 * 16 * 128, BC * 128, 1024), idesc_pv,
+                        (pv_count > 0 || k16 > 0) ? 1u : 0u);
           ++pv_count;
         }
         ssa::mma_commit(smem_u32(&empty_bar[st]));  // the stage is free once these MMAs are done
-        // (S_{t+1} overwrites P_t: it follows the P.V in issue order)
-        if (t + 1 < ntiles) ok = issue_s(t + 1);
+        ssa::mma_commit(smem_u32(&pv_done));        // O holds every P.V up to tile t
+        // (S_{t+2} overwrites P_t: it follows the P.V in issue order)
+        if (t + 2 < ntiles) ok = issue_s(t + 2);
       }
       if (!ok) atomicOr(p.status, 1);
       ssa::mma_commit(smem_u32(&o_done));
@@ -231,7 +239,7 @@ __global__ void __launch_bounds__(NT, 1)
     int n_pv = 0, skipped = 0;
     bool failed = false;
     for (int t = 0; t < ntiles; ++t) {
-      bool ok = !failed && mbar_wait(smem_u32(&s_full), t & 1, p.wait_ns);
+      bool ok = !failed && mbar_wait(smem_u32(&s_full[t & 1]), (t >> 1) & 1, p.wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok && !failed) {
         if (lane == 0) atomicOr(p.status, 1);
@@ -240,7 +248,7 @@ __global__ void __launch_bounds__(NT, 1)
       ssa::tc_fence_after();
       float x[BC];
 #pragma unroll
-      for (int c = 0; c < BC / 32; ++c) ssa::tmem_ld32f(tmem + 32 * c, &x[32 * c]);
+      for (int c = 0; c < BC / 32; ++c) ssa::tmem_ld32f(tmem + s_col(t) + 32 * c, &x[32 * c]);
       ssa::tmem_wait_ld();
       const int j0 = (kt0 + t) * BC;
       int lim = p.Lk - 1 - j0;  // last visible key of this row, relative to the tile
@@ -276,10 +284,18 @@ __global__ void __launch_bounds__(NT, 1)
             __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
             pk[c2] = *reinterpret_cast<uint32_t*>(&pb);
           }
-          ssa::tmem_st32(tmem + 32 * h, pk);
+          ssa::tmem_st32(tmem + s_col(t) + 32 * h, pk);
         }
         if (__any_sync(0xffffffffu, grow) && n_pv > 0) {
-          // every earlier P.V finished before S_t did: rescale O in place
+          // rescale O in place once every earlier P.V has finished (S_t was
+          // issued before the last of them)
+          bool done = !failed && mbar_wait(smem_u32(&pv_done), (t - 1) & 1, p.wait_ns);
+          done = __all_sync(0xffffffffu, done);
+          if (!done && !failed) {
+            if (lane == 0) atomicOr(p.status, 1);
+            failed = true;
+          }
+          ssa::tc_fence_after();
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
