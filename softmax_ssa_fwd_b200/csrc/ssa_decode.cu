@@ -20,8 +20,9 @@
 // 128-row query tile (the rest zero); a key tile is decided per query head
 // (its Lq rows).  160 threads:
 //   warp 0   producer: TMA loads of each key tile's K and V (128-byte swizzled
-//            64-column boxes) into an NS-stage shared-memory ring, up to NS
-//            tiles ahead.  Decode is bound by these bytes, so V is fetched
+//            64-column boxes) into shared-memory rings (3 K tiles, 2 V
+//            tiles: a K tile is free once its S is computed, a V tile only
+//            after its P.V), ahead of the arithmetic.  Decode is bound by these bytes, so V is fetched
 //            with K: a skipped tile saves its exponentials and P.V, not its
 //            V bytes.
 //   warp 1   TMEM owner and MMA issuer: S = Q K^T into TMEM columns [0, Bc),
@@ -54,7 +55,8 @@ using ssa::smem_u32;
 
 constexpr int NT = 160;          // warps 0 producer, 1 MMA, 2-3 idle, 4 softmax
 constexpr int RMAX = 32;         // query rows per CTA: TMEM lanes 0-31, the softmax warp's
-constexpr int NS = 3;            // K/V ring depth (tiles)
+constexpr int KST = 3;           // K ring depth (tiles)
+constexpr int VST = 2;           // V ring depth (tiles)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t O_COL = 128;  // O at TMEM columns [128, 128 + d)
 // S of key tile t (then its P) at columns [256 * (t & 1), 256 * (t & 1) + Bc):
@@ -88,9 +90,9 @@ template <int D, int BC>
 struct DecSmem {
   static constexpr uint32_t Q_BYTES = 128 * D * 2;         // the query tile, rows padded to 128
   static constexpr uint32_t TILE_BYTES = BC * D * 2;        // one K or V tile
-  static constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;   // K then V
-  static constexpr uint32_t RING_BYTES = NS * STAGE_BYTES;
-  static constexpr uint32_t TOTAL = 1024 + Q_BYTES + RING_BYTES;  // + alignment slack
+  static constexpr uint32_t K_OFF = Q_BYTES;
+  static constexpr uint32_t V_OFF = K_OFF + KST * TILE_BYTES;
+  static constexpr uint32_t TOTAL = 1024 + V_OFF + VST * TILE_BYTES;  // + alignment slack
 };
 
 template <int D, int BC>
@@ -100,8 +102,7 @@ __global__ void __launch_bounds__(NT, 1)
   using L = DecSmem<D, BC>;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* q_tile = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = q_tile + L::Q_BYTES;
-  __shared__ uint64_t full_bar[NS], empty_bar[NS];
+  __shared__ uint64_t kfull[KST], kempty[KST], vfull[VST], vempty[VST];
   __shared__ uint64_t s_full[2], p_ready, pv_done, o_done, mma_done;
   __shared__ uint32_t tmem_base;
   __shared__ uint32_t keep_word;
@@ -114,9 +115,13 @@ __global__ void __launch_bounds__(NT, 1)
   const int ntiles = max(0, kt1 - kt0);
 
   if (tid == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(smem_u32(&full_bar[i]), 1);
-      mbar_init(smem_u32(&empty_bar[i]), 1);
+    for (int i = 0; i < KST; ++i) {
+      mbar_init(smem_u32(&kfull[i]), 1);
+      mbar_init(smem_u32(&kempty[i]), 1);
+    }
+    for (int i = 0; i < VST; ++i) {
+      mbar_init(smem_u32(&vfull[i]), 1);
+      mbar_init(smem_u32(&vempty[i]), 1);
     }
     mbar_init(smem_u32(&s_full[0]), 1);
     mbar_init(smem_u32(&s_full[1]), 1);
@@ -147,7 +152,7 @@ __global__ void __launch_bounds__(NT, 1)
   __syncthreads();
   ssa::tc_fence_after();
   const uint32_t tmem = tmem_base;
-  const uint32_t q_s = smem_u32(q_tile), ring_s = smem_u32(ring);
+  const uint32_t q_s = smem_u32(q_tile), k_ring = q_s + L::K_OFF, v_ring = q_s + L::V_OFF;
 
   if (warp == 0) {
     // ======================= producer: K and V tiles by TMA =======================
@@ -156,25 +161,38 @@ __global__ void __launch_bounds__(NT, 1)
       ssa::tma_prefetch_desc(&tm_v);
       int issued = 0;
       for (int t = 0; t < ntiles; ++t) {
-        const int st = t % NS;
-        if (!mbar_wait(smem_u32(&empty_bar[st]), ((t / NS) & 1) ^ 1, p.wait_ns)) {
+        const int j0 = (kt0 + t) * BC;
+        const int ks = t % KST, vs = t % VST;
+        if (!mbar_wait(smem_u32(&kempty[ks]), ((t / KST) & 1) ^ 1, p.wait_ns)) {
           atomicOr(p.status, 1);
           break;
         }
-        const uint32_t fb = smem_u32(&full_bar[st]);
-        mbar_arrive_expect_tx(fb, L::STAGE_BYTES);
-        const uint32_t kd = ring_s + st * L::STAGE_BYTES, vd = kd + L::TILE_BYTES;
-        const int j0 = (kt0 + t) * BC;
+        const uint32_t kb = smem_u32(&kfull[ks]);
+        mbar_arrive_expect_tx(kb, L::TILE_BYTES);
 #pragma unroll
-        for (int box = 0; box < D / 64; ++box) {
-          ssa::tma_load_4d(kd + box * BC * 128, &tm_k, fb, box * 64, hkv, j0, b);
-          ssa::tma_load_4d(vd + box * BC * 128, &tm_v, fb, box * 64, hkv, j0, b);
+        for (int box = 0; box < D / 64; ++box)
+          ssa::tma_load_4d(k_ring + ks * L::TILE_BYTES + box * BC * 128, &tm_k, kb, box * 64, hkv, j0, b);
+        if (!mbar_wait(smem_u32(&vempty[vs]), ((t / VST) & 1) ^ 1, p.wait_ns)) {
+          atomicOr(p.status, 1);
+          // the K load of this tile is in flight: wait for it below
+          issued = -(t + 1);
+          break;
         }
+        const uint32_t vb = smem_u32(&vfull[vs]);
+        mbar_arrive_expect_tx(vb, L::TILE_BYTES);
+#pragma unroll
+        for (int box = 0; box < D / 64; ++box)
+          ssa::tma_load_4d(v_ring + vs * L::TILE_BYTES + box * BC * 128, &tm_v, vb, box * 64, hkv, j0, b);
         issued = t + 1;
       }
-      bool drained = true;  // every load issued has landed before the CTA may exit
-      for (int t = max(0, issued - NS); t < issued; ++t)
-        drained &= mbar_wait(smem_u32(&full_bar[t % NS]), (t / NS) & 1, DRAIN_NS);
+      // drain: every load issued has landed before the CTA may exit
+      bool drained = true;
+      const int kdone = issued < 0 ? -issued : issued;  // K tiles issued
+      const int vdone = issued < 0 ? -issued - 1 : issued;  // V tiles issued
+      for (int t = max(0, kdone - KST); t < kdone; ++t)
+        drained &= mbar_wait(smem_u32(&kfull[t % KST]), (t / KST) & 1, DRAIN_NS);
+      for (int t = max(0, vdone - VST); t < vdone; ++t)
+        drained &= mbar_wait(smem_u32(&vfull[t % VST]), (t / VST) & 1, DRAIN_NS);
       if (!drained) atomicOr(p.status, 1);
     }
   } else if (warp == 1) {
@@ -184,10 +202,10 @@ __global__ void __launch_bounds__(NT, 1)
       constexpr uint32_t idesc_pv = ssa::idesc_bf16_f32(128, D, false, true);
       // S_t = Q K_t^T into TMEM columns [s_col(t), s_col(t) + BC)
       auto issue_s = [&](int t) -> bool {
-        const int st = t % NS;
-        if (!mbar_wait(smem_u32(&full_bar[st]), (t / NS) & 1, p.wait_ns)) return false;
+        const int ks = t % KST;
+        if (!mbar_wait(smem_u32(&kfull[ks]), (t / KST) & 1, p.wait_ns)) return false;
         ssa::tc_fence_after();
-        const uint32_t k_s = ring_s + st * L::STAGE_BYTES;
+        const uint32_t k_s = k_ring + ks * L::TILE_BYTES;
 #pragma unroll
         for (int k16 = 0; k16 < D / 16; ++k16) {
           const uint32_t qoff = (k16 >> 2) * (128 * 128) + (k16 & 3) * 32;
@@ -196,21 +214,27 @@ __global__ void __launch_bounds__(NT, 1)
                       ssa::smem_desc_sw128(k_s + koff, 16, 1024), idesc_qk, k16 > 0 ? 1u : 0u);
         }
         ssa::mma_commit(smem_u32(&s_full[t & 1]));
+        ssa::mma_commit(smem_u32(&kempty[ks]));  // the K tile is free once S_t is done
         return true;
       };
       bool ok = issue_s(0);
       if (ok && ntiles > 1) ok = issue_s(1);
       int pv_count = 0;
       for (int t = 0; ok && t < ntiles; ++t) {
-        const int st = t % NS;
+        const int vs = t % VST;
         if (!mbar_wait(smem_u32(&p_ready), t & 1, p.wait_ns)) {
+          ok = false;
+          break;
+        }
+        // the V tile has to have landed before its slot is handed back, kept or not
+        if (!mbar_wait(smem_u32(&vfull[vs]), (t / VST) & 1, p.wait_ns)) {
           ok = false;
           break;
         }
         if (*reinterpret_cast<volatile uint32_t*>(&keep_word)) {
           // O += P V: P (bf16 pairs over the S columns) from TMEM, V from the stage
           ssa::tc_fence_after();
-          const uint32_t v_s = ring_s + st * L::STAGE_BYTES + L::TILE_BYTES;
+          const uint32_t v_s = v_ring + vs * L::TILE_BYTES;
 #pragma unroll
           for (int k16 = 0; k16 < BC / 16; ++k16)
             ssa::mma_ts(tmem + O_COL, tmem + s_col(t) + k16 * 8,
@@ -218,7 +242,7 @@ __global__ void __launch_bounds__(NT, 1)
                         (pv_count > 0 || k16 > 0) ? 1u : 0u);
           ++pv_count;
         }
-        ssa::mma_commit(smem_u32(&empty_bar[st]));  // the stage is free once these MMAs are done
+        ssa::mma_commit(smem_u32(&vempty[vs]));  // the V tile is free once these MMAs are done
         ssa::mma_commit(smem_u32(&pv_done));        // O holds every P.V up to tile t
         // (S_{t+2} overwrites P_t: it follows the P.V in issue order)
         if (t + 2 < ntiles) ok = issue_s(t + 2);
