@@ -1,5 +1,6 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA tiled
-// loads, tcgen05 (TMEM alloc, MMA, commit, ld/st, fences) and named barriers.
+// loads, tcgen05 (TMEM alloc, MMA, commit, ld/st, fences), shared-memory
+// accesses and packed fp32 arithmetic.
 //
 // Encodings of the two tcgen05 descriptors follow the public PTX ISA
 // ("Matrix Descriptors" / "Instruction descriptor" for tcgen05.mma): the
@@ -107,11 +108,7 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// ---------------------------------------------------------------- barriers
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
+// ---------------------------------------------------------------- shared memory
 // Plain shared-memory accesses that the compiler may not cache or reorder
 // across the surrounding mbarrier operations.
 __device__ __forceinline__ void st_shared_u8(uint32_t addr, uint32_t v) {
@@ -240,11 +237,6 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
 __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 // three-input max

@@ -61,11 +61,6 @@ constexpr uint64_t DRAIN_TIMEOUT_NS = 2000000000ull;
 constexpr float RESCALE_LOG2 = 8.0f;  // lazy O rescale once the max grew by 2^8
 // Key tiles a CTA can list when the caller selects key blocks by bitmap.
 constexpr int MAX_LISTED_TILES = 2048;
-// When POLY_EVERY > 0, one exp2 pair in POLY_EVERY runs as a polynomial on
-// the FMA pipe instead of the MUFU unit.  Measured on B200 (llama8k, wan) the
-// softmax here is latency-bound, not MUFU-bound, and every offload ratio
-// tried (1/2, 1/3, 1/4, 1/8) was slower than none, so it is off.
-constexpr int POLY_EVERY = 0;
 
 struct Params {
   __nv_bfloat16* out;
@@ -134,29 +129,6 @@ __device__ __forceinline__ float mufu_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA pipe: x = n + f with n = rint(x) (by the 1.5 * 2^23 shift),
-// f in [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial (max relative error
-// 7.5e-5, below bf16 resolution; coefficients from csrc/fit_exp2_poly.py);
-// 2^n by adding n to the exponent field.  Arguments below -126 give 0.
-__device__ __forceinline__ float2 poly_exp2x2(uint64_t x01) {
-  constexpr float SHIFT = 12582912.0f;  // 1.5 * 2^23
-  constexpr float C0 = 0x1.fff692p-1f, C1 = 0x1.62f31ap-1f, C2 = 0x1.f0de1ap-3f, C3 = 0x1.c3f76p-5f;
-  float x0, x1;
-  f2_unpack(x01, x0, x1);
-  const uint64_t a = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
-  const uint64_t r = fadd2(a, f2_pack(SHIFT, SHIFT));            // round to nearest integer
-  const uint64_t f = fsub2(a, fsub2(r, f2_pack(SHIFT, SHIFT)));  // fraction in [-1/2, 1/2]
-  uint64_t q = ffma2(f2_pack(C3, C3), f, f2_pack(C2, C2));
-  q = ffma2(q, f, f2_pack(C1, C1));
-  q = ffma2(q, f, f2_pack(C0, C0));
-  float q0, q1, r0, r1;
-  f2_unpack(q, q0, q1);
-  f2_unpack(r, r0, r1);
-  const uint32_t b0 = __float_as_uint(q0) + (__float_as_uint(r0) << 23);
-  const uint32_t b1 = __float_as_uint(q1) + (__float_as_uint(r1) << 23);
-  return make_float2(x0 < -126.f ? 0.f : __uint_as_float(b0), x1 < -126.f ? 0.f : __uint_as_float(b1));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -516,17 +488,9 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const uint64_t a2 = ffma2(f2_pack(x[64 * bb + 2 * i], x[64 * bb + 2 * i + 1]), c2, nm2);
-          float p0, p1;
-          if (POLY_EVERY > 0 && (i % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1) {
-            const float2 ev = poly_exp2x2(a2);
-            p0 = ev.x;
-            p1 = ev.y;
-          } else {
-            float a0, a1;
-            f2_unpack(a2, a0, a1);
-            p0 = mufu_exp2(a0);
-            p1 = mufu_exp2(a1);
-          }
+          float a0, a1;
+          f2_unpack(a2, a0, a1);
+          const float p0 = mufu_exp2(a0), p1 = mufu_exp2(a1);
           ls2 = fadd2(ls2, f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
