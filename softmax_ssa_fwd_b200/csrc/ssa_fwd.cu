@@ -87,7 +87,7 @@ struct __align__(8) Bars {
   uint64_t q_full;
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
-  uint64_t s_full[NQT], p_ready[NQT], o_done[NQT];
+  uint64_t s_full[NQT], p_half[NQT], p_ready[NQT], o_done[NQT];
   uint64_t vote_bar[NQT][2];  // per tile, per step parity: one arrival per softmax warp
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -458,6 +458,21 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     // nothing: the exponentials may start before the vote completes.  A
     // tile right after a skipped one waits for the vote instead, so long
     // runs of skipped tiles spend no MUFU time.
+    // P of every row for this key tile
+    auto store_zero_p = [&]() {
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) pk[i] = 0u;
+#pragma unroll
+      for (int h = 0; h < BC / 64; ++h) tmem_st32(lane_base + s_col + 32 * h, pk);
+    };
+    // "P of the first 64 keys is in TMEM" (one arrival per warp, every step)
+    auto send_first_half = [&]() {
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_half[t]));
+    };
     bool decided = !vote_on;
     if (!decided && !(spec_ok && prev_keep)) {
       decide();
@@ -469,8 +484,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       float m_ref_new = m_ref, alpha = 1.f;
       if (m_ref == -INFINITY) m_ref_new = m_new;  // first kept key: O and l are still zero
       else resc = (m_new - m_ref) * p.scale_log2 > RESCALE_LOG2;
-      // O is rescaled after P is written (the S registers are free then);
-      // every earlier P.V of this tile completed before S(j) did.
+      // O, when rescaled, is rescaled before this tile's P.V may start.
       const bool any_resc = __any_sync(0xffffffffu, resc);
       if (resc) {
         alpha = mufu_exp2((m_ref - m_new) * p.scale_log2);
@@ -482,8 +496,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       const float mref_s = (m_ref_new == -INFINITY) ? 0.f : m_ref_new * c;
       const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-mref_s, -mref_s);
       uint64_t ls2 = f2_pack(0.f, 0.f);
-#pragma unroll
-      for (int bb = 0; bb < BC / 64; ++bb) {
+      auto p_block = [&](int bb) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -495,16 +508,16 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st32(lane_base + s_col + 32 * bb, pk);
-      }
+      };
+      // the first 64 keys' P, then the decision; the MMA warp may start the
+      // P.V on those keys while the rest of P is computed
+      p_block(0);
       if (!decided) decide();
       const bool mine = half ? keep_h[1] : keep_h[0];
       if (mine) {
-        float ls0, ls1;
-        f2_unpack(ls2, ls0, ls1);
-        l = l * alpha + (ls0 + ls1);
-        m_true = m_new;
-        m_ref = m_ref_new;
         if (any_resc && n_pv > 0) {
+          // O must be final before this tile's P.V starts (every earlier P.V
+          // of this tile completed before S(j) did)
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
@@ -518,19 +531,23 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       } else if (keep_h[0] || keep_h[1]) {
         // speculated, and only the other half of a 64-row pair keeps it
         tmem_wait_st();
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) pk[i] = 0u;
-#pragma unroll
-        for (int h = 0; h < BC / 64; ++h) tmem_st32(lane_base + s_col + 32 * h, pk);
+        store_zero_p();
       }
-    } else if (keep_h[0] || keep_h[1]) {
-      // decided: only the other half of a 64-row pair keeps this key tile
-      uint32_t pk[32];
+      send_first_half();
+      if (mine) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) pk[i] = 0u;
-#pragma unroll
-      for (int h = 0; h < BC / 64; ++h) tmem_st32(lane_base + s_col + 32 * h, pk);
+        for (int bb = 1; bb < BC / 64; ++bb) p_block(bb);
+        float ls0, ls1;
+        f2_unpack(ls2, ls0, ls1);
+        l = l * alpha + (ls0 + ls1);
+        m_true = m_new;
+        m_ref = m_ref_new;
+      }
+    } else {
+      // decided: the tile is skipped, or only the other half of a 64-row
+      // pair keeps it
+      if (keep_h[0] || keep_h[1]) store_zero_p();
+      send_first_half();
     }
     const bool tile_keep = keep_h[0] || keep_h[1];
     const bool my_keep = half ? keep_h[1] : keep_h[0];
@@ -703,6 +720,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(smem_u32(&bars->vote_bar[i][0]), 4);
       mbar_init(smem_u32(&bars->vote_bar[i][1]), 4);
       mbar_init(smem_u32(&bars->p_ready[i]), 4);  // one arrival per softmax warp
+      mbar_init(smem_u32(&bars->p_half[i]), 4);
       mbar_init(smem_u32(&bars->o_done[i]), 1);
     }
     mbar_init(smem_u32(&bars->mma_done), 1);
@@ -855,21 +873,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
           if (j >= wk.nvis_t[t]) continue;
-          if (!mbar_wait_fast(smem_u32(&bars->p_ready[t]), j & 1, p.wait_ns)) { ok = false; break; }
+          // P.V in two parts: the first 64 keys once their P is in TMEM, the
+          // rest when the whole of P is
+          if (!mbar_wait_fast(smem_u32(&bars->p_half[t]), j & 1, p.wait_ns)) { ok = false; break; }
           const bool keep = !vote_on || ld_shared_u32(smem_u32(&bars->vote[t][j & 1])) != 0u;
+          const uint32_t p_tmem = tmem + 256 * t;
+          auto issue_pv = [&](int k0, int k1) {
+            tc_fence_after();
+#pragma unroll
+            for (int s = k0; s < k1; ++s) {
+              const uint64_t bd = smem_desc_sw128(v_s + slot * L::V_BYTES + s * 16 * 128, BC * 128, 1024);
+              mma_ts(tmem + 256 * t + 128, p_tmem + s * 8, bd, idesc_pv, (pv_count[t] > 0 || s > 0) ? 1u : 0u);
+            }
+          };
           if (keep) {
             if (!v_seen) {
               if (!mbar_wait_fast(smem_u32(&bars->v_full[slot]), (j / VST) & 1, p.wait_ns)) { ok = false; break; }
               v_seen = true;
             }
-            tc_fence_after();
-            const uint32_t p_tmem = tmem + 256 * t;
-#pragma unroll
-            for (int s = 0; s < BC / 16; ++s) {
-              const uint64_t bd = smem_desc_sw128(v_s + slot * L::V_BYTES + s * 16 * 128, BC * 128, 1024);
-              mma_ts(tmem + 256 * t + 128, p_tmem + s * 8, bd, idesc_pv,
-                     (pv_count[t] > 0 || s > 0) ? 1u : 0u);
-            }
+            issue_pv(0, 4);
+          }
+          if (!mbar_wait_fast(smem_u32(&bars->p_ready[t]), j & 1, p.wait_ns)) { ok = false; break; }
+          if (keep) {
+            issue_pv(4, BC / 16);
             ++pv_count[t];
             any_pv = true;
           }
