@@ -15,20 +15,25 @@
 // with the usual log-sum-exp rule.  With one split this is exactly the
 // prefill rule for a single query tile.
 //
-// CTA (split s, KV head, batch): the G = Hq / Hkv query heads that share the
-// KV head, Lq rows each, R = G * Lq <= 32 rows in all, stacked as rows of one
-// 128-row query tile (the rest zero); a key tile is decided per query head
-// (its Lq rows).  160 threads:
+// Work item (split s, KV head, batch): the G = Hq / Hkv query heads that
+// share the KV head, Lq rows each, R = G * Lq <= 32 rows in all, stacked as
+// rows of one 128-row query tile (the rest zero); a key tile is decided per
+// query head (its Lq rows).  The kernel is persistent (one CTA per SM, each
+// taking work items round-robin), so the loads of the next split stream in
+// while the current one finishes.  160 threads:
 //   warp 0   producer: TMA loads of each key tile's K and V (128-byte swizzled
 //            64-column boxes) into shared-memory rings (3 K tiles, 2 V
 //            tiles: a K tile is free once its S is computed, a V tile only
-//            after its P.V), ahead of the arithmetic.  Decode is bound by these bytes, so V is fetched
-//            with K: a skipped tile saves its exponentials and P.V, not its
-//            V bytes.
-//   warp 1   TMEM owner and MMA issuer: S = Q K^T into TMEM columns [0, Bc),
-//            O += P V into columns [128, 128 + d) with P read from TMEM, on
-//            tcgen05 (M = 128: the padding rows cost tensor time, which decode
-//            has to spare, and no CUDA-core arithmetic)
+//            after its P.V), ahead of the arithmetic and across splits.
+//            Decode is bound by these bytes, so V is fetched with K: a
+//            skipped tile saves its exponentials and P.V, not its V bytes.
+//   warp 1   TMEM owner and MMA issuer: S = Q K^T into one of two S buffers
+//            in TMEM, O += P V into one of two O buffers (one per split in
+//            flight) with P read from TMEM, on tcgen05 (M = 128: the padding
+//            rows cost tensor time, which decode has to spare, and no
+//            CUDA-core arithmetic)
+//   warps 2-3  query loader: the next split's query rows into the second of
+//            two query tiles in shared memory
 //   warp 4   softmax: lane r = query row r = TMEM lane r: masks, tile row max,
 //            the per-head vote (ballots), P -> TMEM as bf16 pairs, O rescale
 //            when a row's max grows, and the split's (max, sum, accumulator)
@@ -53,15 +58,17 @@ using ssa::mbar_init;
 using ssa::mbar_wait;
 using ssa::smem_u32;
 
-constexpr int NT = 160;          // warps 0 producer, 1 MMA, 2-3 idle, 4 softmax
-constexpr int RMAX = 32;         // query rows per CTA: TMEM lanes 0-31, the softmax warp's
+constexpr int NT = 160;          // warps 0 producer, 1 MMA, 2-3 query loader, 4 softmax
+constexpr int RMAX = 32;         // query rows per split: TMEM lanes 0-31, the softmax warp's
 constexpr int KST = 3;           // K ring depth (tiles)
 constexpr int VST = 2;           // V ring depth (tiles)
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t O_COL = 128;  // O at TMEM columns [128, 128 + d)
-// S of key tile t (then its P) at columns [256 * (t & 1), 256 * (t & 1) + Bc):
-// S_{t+1} is computed while the softmax of tile t runs
-__device__ __forceinline__ uint32_t s_col(int t) { return 256u * (uint32_t)(t & 1); }
+// S of the CTA's g-th key tile (then its P) at columns [256 * (g & 1), + Bc):
+// S_{g+1} is computed while the softmax of tile g runs
+__device__ __forceinline__ uint32_t s_col(int g) { return 256u * (uint32_t)(g & 1); }
+// O of the CTA's n-th split at columns [128 + 256 * (n & 1), + d): the next
+// split accumulates while this one's O is read out
+__device__ __forceinline__ uint32_t o_col(int n) { return 128u + 256u * (uint32_t)(n & 1); }
 constexpr unsigned long long DRAIN_NS = 2000000000ull;
 
 struct Params {
@@ -75,6 +82,7 @@ struct Params {
   int* status;
   unsigned long long wait_ns;
   int B, Hq, Hkv, Lq, Lk, causal, S, nK, tiles_per_split, G, R;
+  int n_items;        // B * Hkv * S splits, handed out round-robin over the CTAs
   float c;            // scale * log2(e)
   float log2_lambda;  // -inf for lambda == 0
 };
@@ -85,34 +93,48 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// One split (work item): key tiles [kt0, kt0 + nt) of KV head hkv of sequence b.
+struct Item {
+  int s, hkv, b, kt0, nt;
+};
+__device__ __forceinline__ Item item_of(const Params& p, int it) {
+  Item w;
+  w.s = it % p.S;
+  const int bh = it / p.S;
+  w.hkv = bh % p.Hkv;
+  w.b = bh / p.Hkv;
+  w.kt0 = w.s * p.tiles_per_split;
+  w.nt = max(0, min(p.nK, w.kt0 + p.tiles_per_split) - w.kt0);
+  return w;
+}
 
 template <int D, int BC>
 struct DecSmem {
-  static constexpr uint32_t Q_BYTES = 128 * D * 2;         // the query tile, rows padded to 128
+  static constexpr uint32_t Q_BYTES = 128 * D * 2;         // one query tile, rows padded to 128
   static constexpr uint32_t TILE_BYTES = BC * D * 2;        // one K or V tile
-  static constexpr uint32_t K_OFF = Q_BYTES;
+  static constexpr uint32_t K_OFF = 2 * Q_BYTES;            // two query tiles: the next split's is loaded early
   static constexpr uint32_t V_OFF = K_OFF + KST * TILE_BYTES;
   static constexpr uint32_t TOTAL = 1024 + V_OFF + VST * TILE_BYTES;  // + alignment slack
 };
 
+// Persistent: CTA c takes splits c, c + gridDim.x, ... in turn.  Every role
+// walks the same sequence of splits; the K/V ring, the S buffers and their
+// barriers run on per-CTA tile counters across splits, so the loads of the
+// next split overlap the end of the current one.
 template <int D, int BC>
 __global__ void __launch_bounds__(NT, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const Params p) {
   using L = DecSmem<D, BC>;
   extern __shared__ uint8_t dsm_raw[];
-  uint8_t* q_tile = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* q_tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t kfull[KST], kempty[KST], vfull[VST], vempty[VST];
-  __shared__ uint64_t s_full[2], p_ready, pv_done, o_done, mma_done;
+  __shared__ uint64_t q_full[2], q_empty[2], s_full[2], p_ready, pv_done, o_done[2], mma_done;
   __shared__ uint32_t tmem_base;
   __shared__ uint32_t keep_word;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int s = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
   const int G = p.G, R = p.R, Lq = p.Lq;
-  const int kt0 = s * p.tiles_per_split;
-  const int kt1 = min(p.nK, kt0 + p.tiles_per_split);
-  const int ntiles = max(0, kt1 - kt0);
 
   if (tid == 0) {
     for (int i = 0; i < KST; ++i) {
@@ -123,11 +145,14 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_init(smem_u32(&vfull[i]), 1);
       mbar_init(smem_u32(&vempty[i]), 1);
     }
-    mbar_init(smem_u32(&s_full[0]), 1);
-    mbar_init(smem_u32(&s_full[1]), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&q_full[i]), 64);  // every thread of the two loader warps
+      mbar_init(smem_u32(&q_empty[i]), 1);
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&o_done[i]), 1);
+    }
     mbar_init(smem_u32(&p_ready), 1);
     mbar_init(smem_u32(&pv_done), 1);
-    mbar_init(smem_u32(&o_done), 1);
     mbar_init(smem_u32(&mma_done), 1);
     ssa::fence_mbar_init();
   }
@@ -135,60 +160,53 @@ __global__ void __launch_bounds__(NT, 1)
     ssa::tmem_alloc(smem_u32(&tmem_base), TMEM_COLS);
     ssa::tmem_relinquish();
   }
-  // the query tile: row r = g * Lq + i (head hkv * G + g, query row i), rows
-  // R..127 zero; K-major with 128-byte swizzle, as the MMA's A operand
-  for (int e = tid; e < 128 * (D / 8); e += NT) {
-    const int r = e / (D / 8), u = e % (D / 8);
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (r < R) {
-      const int g = r / Lq, i = r % Lq;
-      val = *reinterpret_cast<const uint4*>(p.q + (((size_t)b * Lq + i) * p.Hq + hkv * G + g) * D + 8 * u);
-    }
-    const int box = u >> 3, unit = u & 7;
-    *reinterpret_cast<uint4*>(q_tile + box * 128 * 128 + r * 128 + ((unit ^ (r & 7)) << 4)) = val;
-  }
-  ssa::fence_proxy_async_smem();  // generic writes of the tile, then tensor-core reads
+  // both query tiles zero: rows R..127 stay zero for every split
+  for (int e = tid; e < (int)(2 * L::Q_BYTES / 16); e += NT)
+    reinterpret_cast<uint4*>(q_tiles)[e] = make_uint4(0u, 0u, 0u, 0u);
+  ssa::fence_proxy_async_smem();  // generic writes of the tiles, then tensor-core reads
   ssa::tc_fence_before();
   __syncthreads();
   ssa::tc_fence_after();
   const uint32_t tmem = tmem_base;
-  const uint32_t q_s = smem_u32(q_tile), k_ring = q_s + L::K_OFF, v_ring = q_s + L::V_OFF;
+  const uint32_t q_s = smem_u32(q_tiles), k_ring = q_s + L::K_OFF, v_ring = q_s + L::V_OFF;
 
   if (warp == 0) {
     // ======================= producer: K and V tiles by TMA =======================
-    if (lane == 0 && ntiles > 0) {
+    if (lane == 0) {
       ssa::tma_prefetch_desc(&tm_k);
       ssa::tma_prefetch_desc(&tm_v);
-      int issued = 0;
-      for (int t = 0; t < ntiles; ++t) {
-        const int j0 = (kt0 + t) * BC;
-        const int ks = t % KST, vs = t % VST;
-        if (!mbar_wait(smem_u32(&kempty[ks]), ((t / KST) & 1) ^ 1, p.wait_ns)) {
-          atomicOr(p.status, 1);
-          break;
-        }
-        const uint32_t kb = smem_u32(&kfull[ks]);
-        mbar_arrive_expect_tx(kb, L::TILE_BYTES);
+      int g = 0, kdone = 0, vdone = 0;  // tiles walked; K and V tiles issued
+      bool ok = true;
+      for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
+        const Item w = item_of(p, it);
+        for (int t = 0; t < w.nt; ++t, ++g) {
+          const int j0 = (w.kt0 + t) * BC;
+          const int ks = g % KST, vs = g % VST;
+          if (!mbar_wait(smem_u32(&kempty[ks]), ((g / KST) & 1) ^ 1, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          const uint32_t kb = smem_u32(&kfull[ks]);
+          mbar_arrive_expect_tx(kb, L::TILE_BYTES);
 #pragma unroll
-        for (int box = 0; box < D / 64; ++box)
-          ssa::tma_load_4d(k_ring + ks * L::TILE_BYTES + box * BC * 128, &tm_k, kb, box * 64, hkv, j0, b);
-        if (!mbar_wait(smem_u32(&vempty[vs]), ((t / VST) & 1) ^ 1, p.wait_ns)) {
-          atomicOr(p.status, 1);
-          // the K load of this tile is in flight: wait for it below
-          issued = -(t + 1);
-          break;
-        }
-        const uint32_t vb = smem_u32(&vfull[vs]);
-        mbar_arrive_expect_tx(vb, L::TILE_BYTES);
+          for (int box = 0; box < D / 64; ++box)
+            ssa::tma_load_4d(k_ring + ks * L::TILE_BYTES + box * BC * 128, &tm_k, kb, box * 64, w.hkv, j0, w.b);
+          kdone = g + 1;
+          if (!mbar_wait(smem_u32(&vempty[vs]), ((g / VST) & 1) ^ 1, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          const uint32_t vb = smem_u32(&vfull[vs]);
+          mbar_arrive_expect_tx(vb, L::TILE_BYTES);
 #pragma unroll
-        for (int box = 0; box < D / 64; ++box)
-          ssa::tma_load_4d(v_ring + vs * L::TILE_BYTES + box * BC * 128, &tm_v, vb, box * 64, hkv, j0, b);
-        issued = t + 1;
+          for (int box = 0; box < D / 64; ++box)
+            ssa::tma_load_4d(v_ring + vs * L::TILE_BYTES + box * BC * 128, &tm_v, vb, box * 64, w.hkv, j0, w.b);
+          vdone = g + 1;
+        }
       }
+      if (!ok) atomicOr(p.status, 1);
       // drain: every load issued has landed before the CTA may exit
       bool drained = true;
-      const int kdone = issued < 0 ? -issued : issued;  // K tiles issued
-      const int vdone = issued < 0 ? -issued - 1 : issued;  // V tiles issued
       for (int t = max(0, kdone - KST); t < kdone; ++t)
         drained &= mbar_wait(smem_u32(&kfull[t % KST]), (t / KST) & 1, DRAIN_NS);
       for (int t = max(0, vdone - VST); t < vdone; ++t)
@@ -197,37 +215,60 @@ __global__ void __launch_bounds__(NT, 1)
     }
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
-    if (lane == 0 && ntiles > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_qk = ssa::idesc_bf16_f32(128, BC, false, false);
       constexpr uint32_t idesc_pv = ssa::idesc_bf16_f32(128, D, false, true);
-      // S_t = Q K_t^T into TMEM columns [s_col(t), s_col(t) + BC)
-      auto issue_s = [&](int t) -> bool {
-        const int ks = t % KST;
-        if (!mbar_wait(smem_u32(&kfull[ks]), (t / KST) & 1, p.wait_ns)) return false;
+      // cursor of the S stream: split it_s (its n_s-th non-empty one), its tile t_s; g_s tiles so far
+      int it_s = blockIdx.x, t_s = 0, n_s = 0, g_s = 0;
+      Item w_s{};
+      auto seek = [&](int& it, Item& w) {
+        for (; it < p.n_items; it += gridDim.x) {
+          w = item_of(p, it);
+          if (w.nt > 0) break;
+        }
+      };
+      seek(it_s, w_s);
+      // S_g = Q K_g^T into TMEM columns [s_col(g), s_col(g) + BC)
+      auto issue_s = [&]() -> bool {
+        const int qb = n_s & 1;
+        if (t_s == 0 && !mbar_wait(smem_u32(&q_full[qb]), (n_s >> 1) & 1, p.wait_ns)) return false;
+        const int ks = g_s % KST;
+        if (!mbar_wait(smem_u32(&kfull[ks]), (g_s / KST) & 1, p.wait_ns)) return false;
         ssa::tc_fence_after();
-        const uint32_t k_s = k_ring + ks * L::TILE_BYTES;
+        const uint32_t k_s = k_ring + ks * L::TILE_BYTES, qt = q_s + qb * L::Q_BYTES;
 #pragma unroll
         for (int k16 = 0; k16 < D / 16; ++k16) {
           const uint32_t qoff = (k16 >> 2) * (128 * 128) + (k16 & 3) * 32;
           const uint32_t koff = (k16 >> 2) * (BC * 128) + (k16 & 3) * 32;
-          ssa::mma_ss(tmem + s_col(t), ssa::smem_desc_sw128(q_s + qoff, 16, 1024),
+          ssa::mma_ss(tmem + s_col(g_s), ssa::smem_desc_sw128(qt + qoff, 16, 1024),
                       ssa::smem_desc_sw128(k_s + koff, 16, 1024), idesc_qk, k16 > 0 ? 1u : 0u);
         }
-        ssa::mma_commit(smem_u32(&s_full[t & 1]));
-        ssa::mma_commit(smem_u32(&kempty[ks]));  // the K tile is free once S_t is done
+        ssa::mma_commit(smem_u32(&s_full[g_s & 1]));
+        ssa::mma_commit(smem_u32(&kempty[ks]));  // the K tile is free once S_g is done
+        if (++t_s == w_s.nt) {
+          ssa::mma_commit(smem_u32(&q_empty[qb]));  // and the query tile after the split's last S
+          t_s = 0;
+          ++n_s;
+          it_s += gridDim.x;
+          seek(it_s, w_s);
+        }
+        ++g_s;
         return true;
       };
-      bool ok = issue_s(0);
-      if (ok && ntiles > 1) ok = issue_s(1);
-      int pv_count = 0;
-      for (int t = 0; ok && t < ntiles; ++t) {
-        const int vs = t % VST;
-        if (!mbar_wait(smem_u32(&p_ready), t & 1, p.wait_ns)) {
+      bool ok = true;
+      for (int i = 0; ok && i < 2 && it_s < p.n_items; ++i) ok = issue_s();
+      // cursor of the P.V stream
+      int it_p = blockIdx.x, t_p = 0, n_p = 0, g_p = 0, pv_count = 0;
+      Item w_p{};
+      seek(it_p, w_p);
+      while (ok && it_p < p.n_items) {
+        const int vs = g_p % VST;
+        if (!mbar_wait(smem_u32(&p_ready), g_p & 1, p.wait_ns)) {
           ok = false;
           break;
         }
         // the V tile has to have landed before its slot is handed back, kept or not
-        if (!mbar_wait(smem_u32(&vfull[vs]), (t / VST) & 1, p.wait_ns)) {
+        if (!mbar_wait(smem_u32(&vfull[vs]), (g_p / VST) & 1, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -237,20 +278,57 @@ __global__ void __launch_bounds__(NT, 1)
           const uint32_t v_s = v_ring + vs * L::TILE_BYTES;
 #pragma unroll
           for (int k16 = 0; k16 < BC / 16; ++k16)
-            ssa::mma_ts(tmem + O_COL, tmem + s_col(t) + k16 * 8,
+            ssa::mma_ts(tmem + o_col(n_p), tmem + s_col(g_p) + k16 * 8,
                         ssa::smem_desc_sw128(v_s + k16 * 16 * 128, BC * 128, 1024), idesc_pv,
                         (pv_count > 0 || k16 > 0) ? 1u : 0u);
           ++pv_count;
         }
         ssa::mma_commit(smem_u32(&vempty[vs]));  // the V tile is free once these MMAs are done
-        ssa::mma_commit(smem_u32(&pv_done));        // O holds every P.V up to tile t
-        // (S_{t+2} overwrites P_t: it follows the P.V in issue order)
-        if (t + 2 < ntiles) ok = issue_s(t + 2);
+        ssa::mma_commit(smem_u32(&pv_done));     // O holds every P.V up to this tile
+        if (++t_p == w_p.nt) {
+          // the split's O is complete (the softmax read the previous O in
+          // this buffer before it handed over any P of this split)
+          ssa::mma_commit(smem_u32(&o_done[n_p & 1]));
+          t_p = 0;
+          pv_count = 0;
+          ++n_p;
+          it_p += gridDim.x;
+          seek(it_p, w_p);
+        }
+        ++g_p;
+        // (S_{g+2} overwrites P_g: it follows the P.V in issue order)
+        if (it_s < p.n_items) ok = issue_s();
       }
       if (!ok) atomicOr(p.status, 1);
-      ssa::mma_commit(smem_u32(&o_done));
       ssa::mma_commit(smem_u32(&mma_done));
       if (!mbar_wait(smem_u32(&mma_done), 0, DRAIN_NS)) atomicOr(p.status, 1);
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ======================= query loader: the next split's rows =======================
+    // row r = g * Lq + i (head hkv * G + g, query row i), K-major with 128-byte
+    // swizzle, as the MMA's A operand
+    const int lt = tid - 64;
+    int n = 0;
+    for (int it = blockIdx.x; it < p.n_items; it += gridDim.x) {
+      const Item w = item_of(p, it);
+      if (w.nt == 0) continue;
+      const int qb = n & 1;
+      if (!mbar_wait(smem_u32(&q_empty[qb]), ((n >> 1) & 1) ^ 1, p.wait_ns)) {
+        if (lt == 0) atomicOr(p.status, 1);
+        break;
+      }
+      uint8_t* qt = q_tiles + qb * L::Q_BYTES;
+      for (int e = lt; e < R * (D / 8); e += 64) {
+        const int r = e / (D / 8), u = e % (D / 8);
+        const int g = r / Lq, i = r % Lq;
+        const uint4 val =
+            *reinterpret_cast<const uint4*>(p.q + (((size_t)w.b * Lq + i) * p.Hq + w.hkv * G + g) * D + 8 * u);
+        const int box = u >> 3, unit = u & 7;
+        *reinterpret_cast<uint4*>(qt + box * 128 * 128 + r * 128 + ((unit ^ (r & 7)) << 4)) = val;
+      }
+      ssa::fence_proxy_async_smem();
+      mbar_arrive(smem_u32(&q_full[qb]));
+      ++n;
     }
   } else if (warp == 4) {
     // ======================= softmax: lane r = query row r = TMEM lane r =======================
@@ -259,121 +337,132 @@ __global__ void __launch_bounds__(NT, 1)
     const int g = valid ? r / Lq : 0, i = valid ? r % Lq : 0;
     const int pos = i + p.Lk - Lq;
     const uint32_t head_mask = ((Lq >= 32) ? 0xffffffffu : ((1u << Lq) - 1u)) << ((lane < G ? lane : 0) * Lq);
-    float m_true = -INFINITY, l = 0.f;  // log2 units of scale * q.k
-    int n_pv = 0, skipped = 0;
+    int gt = 0, n = 0;  // tiles and non-empty splits so far
     bool failed = false;
-    for (int t = 0; t < ntiles; ++t) {
-      bool ok = !failed && mbar_wait(smem_u32(&s_full[t & 1]), (t >> 1) & 1, p.wait_ns);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok && !failed) {
+    for (int it = blockIdx.x; it < p.n_items; it += gridDim.x) {
+      const Item w = item_of(p, it);
+      const uint32_t oc = o_col(n);
+      float m_true = -INFINITY, l = 0.f;  // log2 units of scale * q.k
+      int n_pv = 0, skipped = 0;
+      for (int t = 0; t < w.nt; ++t, ++gt) {
+        bool ok = !failed && mbar_wait(smem_u32(&s_full[gt & 1]), (gt >> 1) & 1, p.wait_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok && !failed) {
+          if (lane == 0) atomicOr(p.status, 1);
+          failed = true;
+        }
+        ssa::tc_fence_after();
+        float x[BC];
+#pragma unroll
+        for (int c = 0; c < BC / 32; ++c) ssa::tmem_ld32f(tmem + s_col(gt) + 32 * c, &x[32 * c]);
+        ssa::tmem_wait_ld();
+        const int j0 = (w.kt0 + t) * BC;
+        int lim = p.Lk - 1 - j0;  // last visible key of this row, relative to the tile
+        if (p.causal && pos - j0 < lim) lim = pos - j0;
+        if (!valid || !ok) lim = -1;
+        float mt = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BC; ++c) {
+          x[c] = (c > lim) ? -INFINITY : x[c] * p.c;
+          mt = fmaxf(mt, x[c]);
+        }
+        const bool neg = mt == -INFINITY || (m_true != -INFINITY && (mt - m_true) < p.log2_lambda);
+        const uint32_t negs = __ballot_sync(0xffffffffu, neg || !valid);
+        // lane g < G holds head g's decision; every row reads its own head's
+        const bool head_keeps = lane < G && (negs & head_mask) != head_mask;
+        const uint32_t keeps = __ballot_sync(0xffffffffu, head_keeps);
+        if (lane < G && !head_keeps) ++skipped;
+        const bool mine = valid && ((keeps >> g) & 1u);
+        if (keeps != 0u) {
+          const float m_new = fmaxf(m_true, mt);
+          const bool grow = mine && m_true != -INFINITY && m_new > m_true;
+          const float alpha = grow ? ex2(m_true - m_new) : 1.f;
+          const float mref = (m_new == -INFINITY) ? 0.f : m_new;
+          float sum = 0.f;
+#pragma unroll
+          for (int h = 0; h < BC / 64; ++h) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int c2 = 0; c2 < 32; ++c2) {
+              const float p0 = mine ? ex2(x[64 * h + 2 * c2] - mref) : 0.f;
+              const float p1 = mine ? ex2(x[64 * h + 2 * c2 + 1] - mref) : 0.f;
+              sum += p0 + p1;
+              __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+              pk[c2] = *reinterpret_cast<uint32_t*>(&pb);
+            }
+            ssa::tmem_st32(tmem + s_col(gt) + 32 * h, pk);
+          }
+          if (__any_sync(0xffffffffu, grow) && n_pv > 0) {
+            // rescale O in place once every earlier P.V has finished (S_g was
+            // issued after the P.V of tile g - 2, so at most tile g - 1's is out)
+            bool done = !failed && mbar_wait(smem_u32(&pv_done), (gt - 1) & 1, p.wait_ns);
+            done = __all_sync(0xffffffffu, done);
+            if (!done && !failed) {
+              if (lane == 0) atomicOr(p.status, 1);
+              failed = true;
+            }
+            ssa::tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              ssa::tmem_ld32(tmem + oc + 32 * cc, o);
+              ssa::tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              ssa::tmem_st32(tmem + oc + 32 * cc, o);
+            }
+          }
+          if (mine) {
+            l = l * alpha + sum;
+            m_true = m_new;
+          }
+          ++n_pv;
+        }
+        ssa::tmem_wait_st();
+        if (lane == 0) *reinterpret_cast<volatile uint32_t*>(&keep_word) = keeps != 0u ? 1u : 0u;
+        ssa::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&p_ready));
+      }
+      // ---- end of the split: the unnormalised accumulator and (max, sum) per row
+      bool okf = true;
+      if (w.nt > 0) {
+        okf = !failed && mbar_wait(smem_u32(&o_done[n & 1]), (n >> 1) & 1, p.wait_ns);
+        ++n;
+      }
+      okf = __all_sync(0xffffffffu, okf) && !failed;
+      if (!okf && !failed) {
         if (lane == 0) atomicOr(p.status, 1);
         failed = true;
       }
       ssa::tc_fence_after();
-      float x[BC];
-#pragma unroll
-      for (int c = 0; c < BC / 32; ++c) ssa::tmem_ld32f(tmem + s_col(t) + 32 * c, &x[32 * c]);
-      ssa::tmem_wait_ld();
-      const int j0 = (kt0 + t) * BC;
-      int lim = p.Lk - 1 - j0;  // last visible key of this row, relative to the tile
-      if (p.causal && pos - j0 < lim) lim = pos - j0;
-      if (!valid || !ok) lim = -1;
-      float mt = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BC; ++c) {
-        x[c] = (c > lim) ? -INFINITY : x[c] * p.c;
-        mt = fmaxf(mt, x[c]);
-      }
-      const bool neg = mt == -INFINITY || (m_true != -INFINITY && (mt - m_true) < p.log2_lambda);
-      const uint32_t negs = __ballot_sync(0xffffffffu, neg || !valid);
-      // lane g < G holds head g's decision; every row reads its own head's
-      const bool head_keeps = lane < G && (negs & head_mask) != head_mask;
-      const uint32_t keeps = __ballot_sync(0xffffffffu, head_keeps);
-      if (lane < G && !head_keeps) ++skipped;
-      const bool mine = valid && ((keeps >> g) & 1u);
-      if (keeps != 0u) {
-        const float m_new = fmaxf(m_true, mt);
-        const bool grow = mine && m_true != -INFINITY && m_new > m_true;
-        const float alpha = grow ? ex2(m_true - m_new) : 1.f;
-        const float mref = (m_new == -INFINITY) ? 0.f : m_new;
-        float sum = 0.f;
-#pragma unroll
-        for (int h = 0; h < BC / 64; ++h) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c2 = 0; c2 < 32; ++c2) {
-            const float p0 = mine ? ex2(x[64 * h + 2 * c2] - mref) : 0.f;
-            const float p1 = mine ? ex2(x[64 * h + 2 * c2 + 1] - mref) : 0.f;
-            sum += p0 + p1;
-            __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-            pk[c2] = *reinterpret_cast<uint32_t*>(&pb);
-          }
-          ssa::tmem_st32(tmem + s_col(t) + 32 * h, pk);
-        }
-        if (__any_sync(0xffffffffu, grow) && n_pv > 0) {
-          // rescale O in place once every earlier P.V has finished (S_t was
-          // issued before the last of them)
-          bool done = !failed && mbar_wait(smem_u32(&pv_done), (t - 1) & 1, p.wait_ns);
-          done = __all_sync(0xffffffffu, done);
-          if (!done && !failed) {
-            if (lane == 0) atomicOr(p.status, 1);
-            failed = true;
-          }
-          ssa::tc_fence_after();
+      const int hq = w.hkv * G + g;
+      float* orow = p.o_part + ((((size_t)w.b * p.Hq + hq) * Lq + i) * p.S + w.s) * D;
 #pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            ssa::tmem_ld32(tmem + O_COL + 32 * cc, o);
-            ssa::tmem_wait_ld();
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        if (okf && n_pv > 0) {
+          ssa::tmem_ld32(tmem + oc + 32 * cc, o);
+          ssa::tmem_wait_ld();
+        } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            ssa::tmem_st32(tmem + O_COL + 32 * cc, o);
-          }
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
         }
-        if (mine) {
-          l = l * alpha + sum;
-          m_true = m_new;
-        }
-        ++n_pv;
-      }
-      ssa::tmem_wait_st();
-      if (lane == 0) *reinterpret_cast<volatile uint32_t*>(&keep_word) = keeps != 0u ? 1u : 0u;
-      ssa::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&p_ready));
-    }
-    // ---- end of the split: the unnormalised accumulator and (max, sum) per row
-    bool okf = true;
-    if (ntiles > 0) okf = mbar_wait(smem_u32(&o_done), 0, p.wait_ns);
-    okf = __all_sync(0xffffffffu, okf) && !failed;
-    if (!okf && lane == 0) atomicOr(p.status, 1);
-    ssa::tc_fence_after();
-    const int hq = hkv * G + g;
-    float* orow = p.o_part + ((((size_t)b * p.Hq + hq) * Lq + i) * p.S + s) * D;
-#pragma unroll 1
-    for (int cc = 0; cc < D / 32; ++cc) {
-      uint32_t o[32];
-      if (okf && n_pv > 0) {
-        ssa::tmem_ld32(tmem + O_COL + 32 * cc, o);
-        ssa::tmem_wait_ld();
-      } else {
+        if (valid) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = 0u;
+          for (int e4 = 0; e4 < 8; ++e4)
+            reinterpret_cast<float4*>(orow + 32 * cc)[e4] =
+                make_float4(__uint_as_float(o[4 * e4]), __uint_as_float(o[4 * e4 + 1]),
+                            __uint_as_float(o[4 * e4 + 2]), __uint_as_float(o[4 * e4 + 3]));
+        }
       }
       if (valid) {
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4)
-          reinterpret_cast<float4*>(orow + 32 * cc)[e4] =
-              make_float4(__uint_as_float(o[4 * e4]), __uint_as_float(o[4 * e4 + 1]),
-                          __uint_as_float(o[4 * e4 + 2]), __uint_as_float(o[4 * e4 + 3]));
+        float* ml = p.ml_part + ((((size_t)w.b * p.Hq + hq) * Lq + i) * p.S + w.s) * 2;
+        ml[0] = m_true;
+        ml[1] = (okf && n_pv > 0) ? l : 0.f;
       }
+      if (lane < G) p.sk_part[((size_t)w.b * p.Hq + w.hkv * G + lane) * p.S + w.s] = skipped;
     }
-    if (valid) {
-      float* ml = p.ml_part + ((((size_t)b * p.Hq + hq) * Lq + i) * p.S + s) * 2;
-      ml[0] = m_true;
-      ml[1] = (okf && n_pv > 0) ? l : 0.f;
-    }
-    if (lane < G) p.sk_part[((size_t)b * p.Hq + hkv * G + lane) * p.S + s] = skipped;
   }
 
   // ---- teardown
@@ -432,7 +521,11 @@ static int launch_bc(const CUtensorMap& mk, const CUtensorMap& mv, const Params&
       return SSA_ERR_CUDA;
     attr_set[dev] = true;
   }
-  decode_split_kernel<D, BC><<<dim3(p.S, p.Hkv, p.B), NT, L::TOTAL, st>>>(mk, mv, p);
+  static int n_sm[64] = {};
+  if (!n_sm[dev] && cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return SSA_ERR_CUDA;
+  const int grid = p.n_items < n_sm[dev] ? p.n_items : n_sm[dev];  // one CTA per SM, persistent
+  decode_split_kernel<D, BC><<<grid, NT, L::TOTAL, st>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return SSA_ERR_CUDA;
   decode_combine_kernel<D><<<dim3(p.Lq, p.Hq, p.B), D / 2, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
@@ -491,6 +584,8 @@ int ssa_decode(const void* q, const void* k, const void* v, void* out, float* ls
   p.S = num_splits;
   p.nK = (Lk + Bc - 1) / Bc;
   p.tiles_per_split = (p.nK + num_splits - 1) / num_splits;
+  if ((long long)B * Hkv * num_splits > (1LL << 30)) return SSA_ERR_UNSUPPORTED;
+  p.n_items = B * Hkv * num_splits;
   p.G = G;
   p.R = G * Lq;
   p.c = (float)((double)scale * 1.4426950408889634);

@@ -68,6 +68,9 @@ CASES = [
     (1, 8, 2, 2, 900, 128, True, 128, 3, 2.0, 12.0),     # lambda > 1
     (1, 4, 2, 1, 200, 128, True, 128, 8, 1e-3, 12.0),    # more splits than key tiles
     (1, 32, 8, 1, 4096, 128, True, 128, 16, 1e-4, 3.0),  # decode shape, literal inputs
+    (4, 32, 8, 1, 2000, 128, True, 64, 40, 1e-3, 12.0),  # more splits than SMs (several per CTA), empty ones
+    (3, 16, 4, 2, 5000, 128, True, 128, 24, 1e-2, 12.0), # several splits per CTA, two query rows
+    (4, 32, 8, 1, 2000, 128, True, 64, 12, 1e-3, 12.0),  # several per CTA, skips inside splits
 ]
 
 
