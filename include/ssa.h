@@ -183,7 +183,8 @@ int ssa_device_status(void* stream);
  *                    summed over splits (overwritten).
  *   workspace:       device scratch of at least ssa_decode_workspace_bytes()
  *                    bytes, 16-byte aligned, owned by the caller; holds the
- *                    per-split partial results between the two kernels.
+ *                    partial results between the two kernels (four per
+ *                    split and query row: accumulator, max and sum).
  *   Limits: d in {64, 128}, Bc in {64, 128}, (Hq / Hkv) * Lq <= 32
  *   (SSA_ERR_UNSUPPORTED otherwise); num_splits >= 1 (splits past the last
  *   key tile are empty and harmless).

@@ -16,11 +16,12 @@
 // prefill rule for a single query tile.
 //
 // Work item (split s, KV head, batch): the G = Hq / Hkv query heads that
-// share the KV head, Lq rows each, R = G * Lq <= 32 rows in all, stacked as
-// rows of one 128-row query tile (the rest zero); a key tile is decided per
-// query head (its Lq rows).  The kernel is persistent (one CTA per SM, each
-// taking work items round-robin), so the loads of the next split stream in
-// while the current one finishes.  160 threads:
+// share the KV head, Lq rows each, R = G * Lq <= 32 rows in all, copied into
+// each of the four 32-row lane quadrants of one 128-row query tile (the rest
+// zero); a key tile is decided per query head (its Lq rows).  The kernel is
+// persistent (one CTA per SM, each taking work items round-robin), so the
+// loads of the next split stream in while the current one finishes.  256
+// threads:
 //   warp 0   producer: TMA loads of each key tile's K and V (128-byte swizzled
 //            64-column boxes) into shared-memory rings (3 K tiles, 2 V
 //            tiles: a K tile is free once its S is computed, a V tile only
@@ -29,14 +30,17 @@
 //            skipped tile saves its exponentials and P.V, not its V bytes.
 //   warp 1   TMEM owner and MMA issuer: S = Q K^T into one of two S buffers
 //            in TMEM, O += P V into one of two O buffers (one per split in
-//            flight) with P read from TMEM, on tcgen05 (M = 128: the padding
-//            rows cost tensor time, which decode has to spare, and no
-//            CUDA-core arithmetic)
+//            flight) with P read from TMEM, on tcgen05 (M = 128: the copies
+//            cost tensor time, which decode has to spare, and no CUDA-core
+//            arithmetic)
 //   warps 2-3  query loader: the next split's query rows into the second of
 //            two query tiles in shared memory
-//   warp 4   softmax: lane r = query row r = TMEM lane r: masks, tile row max,
+//   warps 4-7  softmax, one per lane quadrant, each on a quarter of the key
+//            columns: masks, the tile row max (shared by the four warps),
 //            the per-head vote (ballots), P -> TMEM as bf16 pairs, O rescale
-//            when a row's max grows, and the split's (max, sum, accumulator)
+//            when a row's max grows; each warp's quadrant of O and its row
+//            sums are one partial result of the split, and the combine
+//            kernel merges the four partials of every split with the splits
 // Every wait is bounded; a wait that gives up raises the per-device status
 // word that ssa_device_status reads.
 #include <cuda.h>
@@ -58,8 +62,9 @@ using ssa::mbar_init;
 using ssa::mbar_wait;
 using ssa::smem_u32;
 
-constexpr int NT = 160;          // warps 0 producer, 1 MMA, 2-3 query loader, 4 softmax
-constexpr int RMAX = 32;         // query rows per split: TMEM lanes 0-31, the softmax warp's
+constexpr int NT = 256;          // warps 0 producer, 1 MMA, 2-3 query loader, 4-7 softmax
+constexpr int RMAX = 32;         // query rows per split: one TMEM lane quadrant
+constexpr int NPART = 4;         // partial results per split: one per softmax warp
 constexpr int KST = 3;           // K ring depth (tiles)
 constexpr int VST = 2;           // V ring depth (tiles)
 constexpr uint32_t TMEM_COLS = 512;
@@ -76,8 +81,8 @@ struct Params {
   __nv_bfloat16* out;
   float* lse;
   int32_t* skip_count;
-  float* o_part;    // [B, Hq, Lq, S, d]
-  float* ml_part;   // [B, Hq, Lq, S, 2]: running max (log2 units), row sum
+  float* o_part;    // [B, Hq, Lq, S * NPART, d]
+  float* ml_part;   // [B, Hq, Lq, S * NPART, 2]: running max (log2 units), row sum
   int32_t* sk_part; // [B, Hq, S]
   int* status;
   unsigned long long wait_ns;
@@ -129,9 +134,10 @@ __global__ void __launch_bounds__(NT, 1)
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* q_tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t kfull[KST], kempty[KST], vfull[VST], vempty[VST];
-  __shared__ uint64_t q_full[2], q_empty[2], s_full[2], p_ready, pv_done, o_done[2], mma_done;
+  __shared__ uint64_t q_full[2], q_empty[2], s_full[2], p_ready[2], pv_done, o_done[2], mma_done;
   __shared__ uint32_t tmem_base;
-  __shared__ uint32_t keep_word;
+  __shared__ uint32_t keep_word[2];            // tile decision for the MMA warp, by tile parity
+  __shared__ float red_max[2][4][32];          // per-warp row maxima, by tile parity
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.G, R = p.R, Lq = p.Lq;
@@ -150,8 +156,12 @@ __global__ void __launch_bounds__(NT, 1)
       mbar_init(smem_u32(&q_empty[i]), 1);
       mbar_init(smem_u32(&s_full[i]), 1);
       mbar_init(smem_u32(&o_done[i]), 1);
+      // P of the CTA's tiles 2m + i: one arrival per softmax warp.  One
+      // barrier per tile parity, like S: the softmax can finish tile g + 1
+      // (and, once S_{g+2} is issued, g + 2) before the MMA warp has looked
+      // at tile g + 1's phase
+      mbar_init(smem_u32(&p_ready[i]), 4);
     }
-    mbar_init(smem_u32(&p_ready), 1);
     mbar_init(smem_u32(&pv_done), 1);
     mbar_init(smem_u32(&mma_done), 1);
     ssa::fence_mbar_init();
@@ -263,7 +273,7 @@ __global__ void __launch_bounds__(NT, 1)
       seek(it_p, w_p);
       while (ok && it_p < p.n_items) {
         const int vs = g_p % VST;
-        if (!mbar_wait(smem_u32(&p_ready), g_p & 1, p.wait_ns)) {
+        if (!mbar_wait(smem_u32(&p_ready[g_p & 1]), (g_p >> 1) & 1, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -272,7 +282,7 @@ __global__ void __launch_bounds__(NT, 1)
           ok = false;
           break;
         }
-        if (*reinterpret_cast<volatile uint32_t*>(&keep_word)) {
+        if (*reinterpret_cast<volatile uint32_t*>(&keep_word[g_p & 1])) {
           // O += P V: P (bf16 pairs over the S columns) from TMEM, V from the stage
           ssa::tc_fence_after();
           const uint32_t v_s = v_ring + vs * L::TILE_BYTES;
@@ -305,8 +315,10 @@ __global__ void __launch_bounds__(NT, 1)
     }
   } else if (warp == 2 || warp == 3) {
     // ======================= query loader: the next split's rows =======================
-    // row r = g * Lq + i (head hkv * G + g, query row i), K-major with 128-byte
-    // swizzle, as the MMA's A operand
+    // row r = g * Lq + i (head hkv * G + g, query row i), copied to rows r,
+    // 32 + r, 64 + r and 96 + r (one copy per TMEM lane quadrant, so each
+    // softmax warp sees every row); K-major with 128-byte swizzle, as the
+    // MMA's A operand
     const int lt = tid - 64;
     int n = 0;
     for (int it = blockIdx.x; it < p.n_items; it += gridDim.x) {
@@ -324,19 +336,33 @@ __global__ void __launch_bounds__(NT, 1)
         const uint4 val =
             *reinterpret_cast<const uint4*>(p.q + (((size_t)w.b * Lq + i) * p.Hq + w.hkv * G + g) * D + 8 * u);
         const int box = u >> 3, unit = u & 7;
-        *reinterpret_cast<uint4*>(qt + box * 128 * 128 + r * 128 + ((unit ^ (r & 7)) << 4)) = val;
+#pragma unroll
+        for (int cp = 0; cp < 4; ++cp)  // rows 32 cp + r: same swizzle phase (r & 7)
+          *reinterpret_cast<uint4*>(qt + box * 128 * 128 + (32 * cp + r) * 128 + ((unit ^ (r & 7)) << 4)) = val;
       }
       ssa::fence_proxy_async_smem();
       mbar_arrive(smem_u32(&q_full[qb]));
       ++n;
     }
-  } else if (warp == 4) {
-    // ======================= softmax: lane r = query row r = TMEM lane r =======================
+  } else if (warp >= 4) {
+    // ======================= softmax =======================
+    // Warp 4 + qd owns TMEM lanes [32 qd, 32 qd + 32) (its copy of the query
+    // rows: lane r = row r) and key columns [qd * CW, qd * CW + CW) of every
+    // tile.  The four warps share each row's tile max (so every warp takes
+    // the same skip decisions and uses the same running max), and each keeps
+    // its own row sums and, in its lane quadrant of O, its own accumulator:
+    // the four partial results of a split are merged with the splits.
+    constexpr int CW = BC / 4;
+    const int qd = warp - 4;
+    const uint32_t tq = tmem + ((uint32_t)(32 * qd) << 16);
     const int r = lane;
     const bool valid = r < R;
     const int g = valid ? r / Lq : 0, i = valid ? r % Lq : 0;
     const int pos = i + p.Lk - Lq;
     const uint32_t head_mask = ((Lq >= 32) ? 0xffffffffu : ((1u << Lq) - 1u)) << ((lane < G ? lane : 0) * Lq);
+    uint32_t zero[CW / 2];
+#pragma unroll
+    for (int e = 0; e < CW / 2; ++e) zero[e] = 0u;
     int gt = 0, n = 0;  // tiles and non-empty splits so far
     bool failed = false;
     for (int it = blockIdx.x; it < p.n_items; it += gridDim.x) {
@@ -352,20 +378,25 @@ __global__ void __launch_bounds__(NT, 1)
           failed = true;
         }
         ssa::tc_fence_after();
-        float x[BC];
-#pragma unroll
-        for (int c = 0; c < BC / 32; ++c) ssa::tmem_ld32f(tmem + s_col(gt) + 32 * c, &x[32 * c]);
+        float x[CW];
+        if constexpr (CW == 32) ssa::tmem_ld32f(tq + s_col(gt) + qd * CW, x);
+        else ssa::tmem_ld16f(tq + s_col(gt) + qd * CW, x);
         ssa::tmem_wait_ld();
-        const int j0 = (w.kt0 + t) * BC;
-        int lim = p.Lk - 1 - j0;  // last visible key of this row, relative to the tile
+        const int j0 = (w.kt0 + t) * BC + qd * CW;  // first key of this warp's columns
+        int lim = p.Lk - 1 - j0;  // last visible key of this row, relative to j0
         if (p.causal && pos - j0 < lim) lim = pos - j0;
         if (!valid || !ok) lim = -1;
-        float mt = -INFINITY;
+        float ml = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < BC; ++c) {
+        for (int c = 0; c < CW; ++c) {
           x[c] = (c > lim) ? -INFINITY : x[c] * p.c;
-          mt = fmaxf(mt, x[c]);
+          ml = fmaxf(ml, x[c]);
         }
+        // the row's max over the whole tile: the four warps' maxima
+        volatile float* rm = &red_max[gt & 1][0][0];
+        rm[32 * qd + lane] = ml;
+        ssa::named_bar_sync(1, 128);
+        const float mt = fmaxf(fmaxf(rm[lane], rm[32 + lane]), fmaxf(rm[64 + lane], rm[96 + lane]));
         const bool neg = mt == -INFINITY || (m_true != -INFINITY && (mt - m_true) < p.log2_lambda);
         const uint32_t negs = __ballot_sync(0xffffffffu, neg || !valid);
         // lane g < G holds head g's decision; every row reads its own head's
@@ -379,22 +410,27 @@ __global__ void __launch_bounds__(NT, 1)
           const float alpha = grow ? ex2(m_true - m_new) : 1.f;
           const float mref = (m_new == -INFINITY) ? 0.f : m_new;
           float sum = 0.f;
+          uint32_t pk[CW / 2];
 #pragma unroll
-          for (int h = 0; h < BC / 64; ++h) {
-            uint32_t pk[32];
+          for (int c2 = 0; c2 < CW / 2; ++c2) {
+            const float p0 = mine ? ex2(x[2 * c2] - mref) : 0.f;
+            const float p1 = mine ? ex2(x[2 * c2 + 1] - mref) : 0.f;
+            sum += p0 + p1;
+            __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            pk[c2] = *reinterpret_cast<uint32_t*>(&pb);
+          }
+          // P over the tile's columns (bf16 pairs): this warp's keys, zero for
+          // the other warps' keys
 #pragma unroll
-            for (int c2 = 0; c2 < 32; ++c2) {
-              const float p0 = mine ? ex2(x[64 * h + 2 * c2] - mref) : 0.f;
-              const float p1 = mine ? ex2(x[64 * h + 2 * c2 + 1] - mref) : 0.f;
-              sum += p0 + p1;
-              __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-              pk[c2] = *reinterpret_cast<uint32_t*>(&pb);
-            }
-            ssa::tmem_st32(tmem + s_col(gt) + 32 * h, pk);
+          for (int blk = 0; blk < 4; ++blk) {
+            const uint32_t col = tq + s_col(gt) + blk * (CW / 2);
+            if constexpr (CW == 32) ssa::tmem_st16(col, blk == qd ? pk : zero);
+            else ssa::tmem_st8(col, blk == qd ? pk : zero);
           }
           if (__any_sync(0xffffffffu, grow) && n_pv > 0) {
-            // rescale O in place once every earlier P.V has finished (S_g was
-            // issued after the P.V of tile g - 2, so at most tile g - 1's is out)
+            // rescale this quadrant of O once every earlier P.V has finished
+            // (S_g was issued after the P.V of tile g - 2, so at most tile
+            // g - 1's is out)
             bool done = !failed && mbar_wait(smem_u32(&pv_done), (gt - 1) & 1, p.wait_ns);
             done = __all_sync(0xffffffffu, done);
             if (!done && !failed) {
@@ -405,11 +441,11 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
               uint32_t o[32];
-              ssa::tmem_ld32(tmem + oc + 32 * cc, o);
+              ssa::tmem_ld32(tq + oc + 32 * cc, o);
               ssa::tmem_wait_ld();
 #pragma unroll
               for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              ssa::tmem_st32(tmem + oc + 32 * cc, o);
+              ssa::tmem_st32(tq + oc + 32 * cc, o);
             }
           }
           if (mine) {
@@ -419,12 +455,12 @@ __global__ void __launch_bounds__(NT, 1)
           ++n_pv;
         }
         ssa::tmem_wait_st();
-        if (lane == 0) *reinterpret_cast<volatile uint32_t*>(&keep_word) = keeps != 0u ? 1u : 0u;
+        if (qd == 0 && lane == 0) *reinterpret_cast<volatile uint32_t*>(&keep_word[gt & 1]) = keeps != 0u ? 1u : 0u;
         ssa::tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&p_ready));
+        if (lane == 0) mbar_arrive(smem_u32(&p_ready[gt & 1]));
       }
-      // ---- end of the split: the unnormalised accumulator and (max, sum) per row
+      // ---- end of the split: this warp's unnormalised accumulator and (max, sum) per row
       bool okf = true;
       if (w.nt > 0) {
         okf = !failed && mbar_wait(smem_u32(&o_done[n & 1]), (n >> 1) & 1, p.wait_ns);
@@ -437,12 +473,13 @@ __global__ void __launch_bounds__(NT, 1)
       }
       ssa::tc_fence_after();
       const int hq = w.hkv * G + g;
-      float* orow = p.o_part + ((((size_t)w.b * p.Hq + hq) * Lq + i) * p.S + w.s) * D;
+      const size_t part = (((size_t)w.b * p.Hq + hq) * Lq + i) * ((size_t)p.S * NPART) + (size_t)w.s * NPART + qd;
+      float* orow = p.o_part + part * D;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
         if (okf && n_pv > 0) {
-          ssa::tmem_ld32(tmem + oc + 32 * cc, o);
+          ssa::tmem_ld32(tq + oc + 32 * cc, o);
           ssa::tmem_wait_ld();
         } else {
 #pragma unroll
@@ -457,11 +494,11 @@ __global__ void __launch_bounds__(NT, 1)
         }
       }
       if (valid) {
-        float* ml = p.ml_part + ((((size_t)w.b * p.Hq + hq) * Lq + i) * p.S + w.s) * 2;
-        ml[0] = m_true;
-        ml[1] = (okf && n_pv > 0) ? l : 0.f;
+        float* mlp = p.ml_part + part * 2;
+        mlp[0] = m_true;
+        mlp[1] = (okf && n_pv > 0) ? l : 0.f;
       }
-      if (lane < G) p.sk_part[((size_t)w.b * p.Hq + w.hkv * G + lane) * p.S + w.s] = skipped;
+      if (qd == 0 && lane < G) p.sk_part[((size_t)w.b * p.Hq + w.hkv * G + lane) * p.S + w.s] = skipped;
     }
   }
 
@@ -480,18 +517,19 @@ __global__ void decode_combine_kernel(const Params p) {
   const int i = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
   const int t = threadIdx.x;  // column pair
   const size_t row = ((size_t)b * p.Hq + hq) * p.Lq + i;
-  const float* ml = p.ml_part + row * p.S * 2;
+  const int np = p.S * NPART;  // partial results of this row
+  const float* ml = p.ml_part + row * np * 2;
   float M = -INFINITY;
-  for (int s = 0; s < p.S; ++s)
+  for (int s = 0; s < np; ++s)
     if (ml[2 * s + 1] > 0.f) M = fmaxf(M, ml[2 * s]);
   float L = 0.f, a0 = 0.f, a1 = 0.f;
   if (M != -INFINITY) {
-    for (int s = 0; s < p.S; ++s) {
+    for (int s = 0; s < np; ++s) {
       const float ls = ml[2 * s + 1];
       if (!(ls > 0.f)) continue;
       const float w = ex2(ml[2 * s] - M);
       L += w * ls;
-      const float* o = p.o_part + (row * p.S + s) * D;
+      const float* o = p.o_part + (row * np + s) * D;
       a0 = fmaf(w, o[2 * t], a0);
       a1 = fmaf(w, o[2 * t + 1], a1);
     }
@@ -532,8 +570,8 @@ static int launch_bc(const CUtensorMap& mk, const CUtensorMap& mv, const Params&
 }
 
 static size_t workspace_bytes(int B, int Hq, int Lq, int d, int S) {
-  const size_t rows = (size_t)B * Hq * Lq;
-  return rows * S * d * sizeof(float) + rows * S * 2 * sizeof(float) + (size_t)B * Hq * S * sizeof(int32_t);
+  const size_t rows = (size_t)B * Hq * Lq, parts = (size_t)S * NPART;
+  return rows * parts * d * sizeof(float) + rows * parts * 2 * sizeof(float) + (size_t)B * Hq * S * sizeof(int32_t);
 }
 
 }  // namespace ssa_dec
@@ -573,8 +611,8 @@ int ssa_decode(const void* q, const void* k, const void* v, void* out, float* ls
   p.skip_count = tile_skip_count;
   const size_t rows = (size_t)B * Hq * Lq;
   p.o_part = static_cast<float*>(workspace);
-  p.ml_part = p.o_part + rows * num_splits * d;
-  p.sk_part = reinterpret_cast<int32_t*>(p.ml_part + rows * num_splits * 2);
+  p.ml_part = p.o_part + rows * num_splits * NPART * d;
+  p.sk_part = reinterpret_cast<int32_t*>(p.ml_part + rows * num_splits * NPART * 2);
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;

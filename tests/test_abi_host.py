@@ -134,8 +134,9 @@ def test_decode_unsupported_arguments(ssa, over):
 
 
 def test_decode_workspace_bytes(ssa):
-    # partial accumulators (fp32 d per row and split), (max, sum) per row and split, skip counts
-    assert ssa.ssa_decode_workspace_bytes(8, 32, 1, 128, 16) == 8 * 32 * 16 * (128 * 4 + 8) + 8 * 32 * 16 * 4
+    # four partial results per row and split (fp32 accumulator of d, then
+    # (max, sum)), then the skip counts per (batch, head, split)
+    assert ssa.ssa_decode_workspace_bytes(8, 32, 1, 128, 16) == 8 * 32 * 16 * 4 * (128 * 4 + 8) + 8 * 32 * 16 * 4
     assert ssa.ssa_decode_workspace_bytes(0, 32, 1, 128, 16) == 0
 
 

@@ -32,7 +32,7 @@ def _check(q, k, v, *, causal, scale, lam, Bc, splits, heads=None):
     from softmax_ssa_fwd_b200 import ssa
     out, lse, cnt = ssa.decode(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale, lam=lam,
                                Bc=Bc, num_splits=splits)
-    torch.cuda.synchronize()
+    assert ssa.ssa_device_status() == ssa.SSA_OK  # no bounded wait in the kernels gave up
     ref = decode_oracle(q, k, v, causal=causal, scale=scale, lam=lam, Bc=Bc, num_splits=splits,
                         heads=heads)
     o = out.float().cpu().numpy()
