@@ -511,29 +511,52 @@ __global__ void __launch_bounds__(NT, 1)
   }
 }
 
-// Merge the splits of one (batch, head, query row): block of d/2 threads.
+// Merge the partial results of one (batch, head, query row): S * NPART of
+// them, by the log-sum-exp rule.  2 * d threads: first the largest max among
+// the partials that kept a key (all threads), then four groups of d / 2
+// threads (two columns each) sum every fourth partial, and group 0 adds the
+// four group sums.
 template <int D>
-__global__ void decode_combine_kernel(const Params p) {
+__global__ void __launch_bounds__(2 * D) decode_combine_kernel(const Params p) {
+  constexpr int TPG = D / 2, NG = 4, NW = 2 * D / 32;
+  __shared__ float wmax[NW];
+  __shared__ float gacc[NG][D];
+  __shared__ float gsum[NG];
   const int i = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
-  const int t = threadIdx.x;  // column pair
+  const int tid = threadIdx.x, grp = tid / TPG, t = tid % TPG;
   const size_t row = ((size_t)b * p.Hq + hq) * p.Lq + i;
-  const int np = p.S * NPART;  // partial results of this row
+  const int np = p.S * NPART;
   const float* ml = p.ml_part + row * np * 2;
-  float M = -INFINITY;
-  for (int s = 0; s < np; ++s)
-    if (ml[2 * s + 1] > 0.f) M = fmaxf(M, ml[2 * s]);
+  float mx = -INFINITY;
+  for (int s = tid; s < np; s += 2 * D)
+    if (ml[2 * s + 1] > 0.f) mx = fmaxf(mx, ml[2 * s]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) wmax[tid >> 5] = mx;
+  __syncthreads();
+  float M = wmax[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) M = fmaxf(M, wmax[w]);
+  // a partial that kept no key has l = 0 and an all-zero accumulator
   float L = 0.f, a0 = 0.f, a1 = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < np; ++s) {
-      const float ls = ml[2 * s + 1];
-      if (!(ls > 0.f)) continue;
-      const float w = ex2(ml[2 * s] - M);
-      L += w * ls;
-      const float* o = p.o_part + (row * np + s) * D;
-      a0 = fmaf(w, o[2 * t], a0);
-      a1 = fmaf(w, o[2 * t + 1], a1);
-    }
+  const float* ob = p.o_part + row * (size_t)np * D + 2 * t;
+#pragma unroll 4
+  for (int s = grp; s < np; s += NG) {
+    const float ls = ml[2 * s + 1];
+    const float w = ls > 0.f ? ex2(ml[2 * s] - M) : 0.f;
+    const float2 o = *reinterpret_cast<const float2*>(ob + (size_t)s * D);
+    L = fmaf(w, ls, L);
+    a0 = fmaf(w, o.x, a0);
+    a1 = fmaf(w, o.y, a1);
   }
+  gacc[grp][2 * t] = a0;
+  gacc[grp][2 * t + 1] = a1;
+  if (t == 0) gsum[grp] = L;
+  __syncthreads();
+  if (grp != 0) return;
+  a0 = gacc[0][2 * t] + gacc[1][2 * t] + gacc[2][2 * t] + gacc[3][2 * t];
+  a1 = gacc[0][2 * t + 1] + gacc[1][2 * t + 1] + gacc[2][2 * t + 1] + gacc[3][2 * t + 1];
+  L = gsum[0] + gsum[1] + gsum[2] + gsum[3];
   const float inv = L > 0.f ? 1.f / L : 0.f;
   __nv_bfloat162 res = __floats2bfloat162_rn(a0 * inv, a1 * inv);
   *reinterpret_cast<__nv_bfloat162*>(p.out + (((size_t)b * p.Lq + i) * p.Hq + hq) * D + 2 * t) = res;
@@ -565,7 +588,7 @@ static int launch_bc(const CUtensorMap& mk, const CUtensorMap& mv, const Params&
   const int grid = p.n_items < n_sm[dev] ? p.n_items : n_sm[dev];  // one CTA per SM, persistent
   decode_split_kernel<D, BC><<<grid, NT, L::TOTAL, st>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return SSA_ERR_CUDA;
-  decode_combine_kernel<D><<<dim3(p.Lq, p.Hq, p.B), D / 2, 0, st>>>(p);
+  decode_combine_kernel<D><<<dim3(p.Lq, p.Hq, p.B), 2 * D, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
 }
 
