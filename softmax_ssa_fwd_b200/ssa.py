@@ -178,7 +178,8 @@ def decode(q, k, v, *, causal=True, scale=None, lam=0.0, Bc=128, num_splits=None
 
     q [B, Lq, Hq, d] (a few rows), k/v [B, Lk, Hkv, d] bf16 CUDA tensors.  Returns
     (out [B, Lq, Hq, d] bf16, lse [B, Hq, Lq] fp32, tile_skip_count [B, Hq] int32).
-    num_splits defaults to enough key splits for about two CTAs per SM.
+    num_splits defaults to enough key splits for about two work items per SM (the
+    kernel is persistent: one CTA per SM takes the (split, KV head, sequence) items in turn).
     """
     B, Lq, Hq, d = q.shape
     _, Lk, Hkv, _ = k.shape
