@@ -49,6 +49,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/ssa.h"
 #include "internal.h"
@@ -573,19 +574,30 @@ __global__ void __launch_bounds__(2 * D) decode_combine_kernel(const Params p) {
 template <int D, int BC>
 static int launch_bc(const CUtensorMap& mk, const CUtensorMap& mv, const Params& p, cudaStream_t st) {
   using L = DecSmem<D, BC>;
-  static bool attr_set[64] = {};  // per instance and device, before the first launch there
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SSA_ERR_CUDA;
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(decode_split_kernel<D, BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)L::TOTAL) != cudaSuccess)
-      return SSA_ERR_CUDA;
-    attr_set[dev] = true;
+  int n_sm = 0;
+  {
+    // per instance and device, once before the first launch there; callers may be threads
+    static std::mutex mu;
+    static bool attr_set[64] = {};
+    static int sms[64] = {};
+    std::lock_guard<std::mutex> g(mu);
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(decode_split_kernel<D, BC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)L::TOTAL) != cudaSuccess)
+        return SSA_ERR_CUDA;
+      attr_set[dev] = true;
+    }
+    if (!sms[dev]) {
+      int v = 0;
+      if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+        return SSA_ERR_CUDA;
+      sms[dev] = v;
+    }
+    n_sm = sms[dev];
   }
-  static int n_sm[64] = {};
-  if (!n_sm[dev] && cudaDeviceGetAttribute(&n_sm[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return SSA_ERR_CUDA;
-  const int grid = p.n_items < n_sm[dev] ? p.n_items : n_sm[dev];  // one CTA per SM, persistent
+  const int grid = p.n_items < n_sm ? p.n_items : n_sm;  // one CTA per SM, persistent
   decode_split_kernel<D, BC><<<grid, NT, L::TOTAL, st>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return SSA_ERR_CUDA;
   decode_combine_kernel<D><<<dim3(p.Lq, p.Hq, p.B), 2 * D, 0, st>>>(p);
