@@ -28,31 +28,14 @@ missed phase.
 """
 import random
 
-import pytest
+from protocol_model import Bar, ProtocolError, Sim
 
 KST, VST, NWARP = 3, 2, 4
 
 
-class ProtocolError(AssertionError):
-    pass
-
-
-class Bar:
-    def __init__(self, name, count):
-        self.name, self.count, self.pending, self.phase = name, count, count, 0
-
-    def arrive(self):
-        self.pending -= 1
-        if self.pending < 0:
-            raise ProtocolError(f"{self.name}: more arrivals than expected")
-        if self.pending == 0:
-            self.phase += 1
-            self.pending = self.count
-
-
-class Model:
+class Model(Sim):
     def __init__(self, rng, items, per_parity_p_ready=True):
-        self.rng = rng
+        super().__init__(rng)
         self.items = items  # per split: list of (keep, grow) per tile; [] = empty split
         self.per_parity = per_parity_p_ready
         self.nonempty = [n for n, it in enumerate(items) if it]
@@ -81,20 +64,17 @@ class Model:
         self.q_buf = [None, None]
         self.o_read = {}
         self.keep_word = [None, None]
-        self.queue = []   # tensor pipe: ("op", fn) / ("commit", bar), in order
-        self.tma = []     # loads in flight: (bar, on_land), complete in any order
-        self.nbar_gen, self.nbar_count = 0, 0
 
     # ------------------------------------------------------------ roles
     def producer(self):
         for g in range(len(self.tiles)):
             if g >= KST:
                 yield ("wait", self.kempty[g % KST], g // KST - 1)
-            yield ("do", lambda g=g: self._check(g < KST or self.s_exec[g - KST], f"K slot of tile {g} refilled early"))
+            yield ("do", lambda g=g: self.check(g < KST or self.s_exec[g - KST], f"K slot of tile {g} refilled early"))
             yield ("tma", self.kfull[g % KST], lambda g=g: self.k_slot.__setitem__(g % KST, g))
             if g >= VST:
                 yield ("wait", self.vempty[g % VST], g // VST - 1)
-            yield ("do", lambda g=g: self._check(g < VST or (self.mma_done_tile[g - VST] and (self.pv_exec[g - VST] or not self.keep[g - VST])),
+            yield ("do", lambda g=g: self.check(g < VST or (self.mma_done_tile[g - VST] and (self.pv_exec[g - VST] or not self.keep[g - VST])),
                                               f"V slot of tile {g} refilled early"))
             yield ("tma", self.vfull[g % VST], lambda g=g: self.v_slot.__setitem__(g % VST, g))
 
@@ -108,7 +88,7 @@ class Model:
     def _write_q(self, i):
         if i >= 2:
             prev = [g for g, (n, t) in enumerate(self.tiles) if n == self.nonempty[i - 2]]
-            self._check(all(self.s_exec[g] for g in prev), f"query tile of split {i} written before S of split {i - 2} ran")
+            self.check(all(self.s_exec[g] for g in prev), f"query tile of split {i} written before S of split {i - 2} ran")
         self.q_buf[i % 2] = i
 
     def mma(self):
@@ -142,7 +122,7 @@ class Model:
                 yield ("wait", self.p_ready[0], g)
             yield ("wait", self.vfull[g % VST], g // VST)
             kw = self.keep_word[g % 2]
-            self._check(kw is not None and kw[0] == g, f"MMA read the keep flag of tile {kw and kw[0]} for tile {g}")
+            self.check(kw is not None and kw[0] == g, f"MMA read the keep flag of tile {kw and kw[0]} for tile {g}")
             if kw[1]:
                 yield ("op", lambda g=g, i=i, first=(pv_count == 0): self._exec_pv(g, i, first))
                 pv_count += 1
@@ -183,112 +163,39 @@ class Model:
                 i += 1
 
     # ------------------------------------------------------------ checks run by the pipe and the roles
-    def _check(self, ok, what):
-        if not ok:
-            raise ProtocolError(what)
-
     def _exec_s(self, g, i):
         n, t = self.tiles[g]
-        self._check(self.k_slot[g % KST] == g, f"S_{g} read a K slot holding tile {self.k_slot[g % KST]}")
-        self._check(self.q_buf[i % 2] == i, f"S_{g} read the query tile of split {self.q_buf[i % 2]}")
+        self.check(self.k_slot[g % KST] == g, f"S_{g} read a K slot holding tile {self.k_slot[g % KST]}")
+        self.check(self.q_buf[i % 2] == i, f"S_{g} read the query tile of split {self.q_buf[i % 2]}")
         if g >= 2:
-            self._check(self.s_read[g - 2] == NWARP, f"S_{g} overwrote S_{g - 2} before every warp read it")
-            self._check(self.pv_exec[g - 2] or not self.keep[g - 2], f"S_{g} overwrote P_{g - 2} before its P.V")
+            self.check(self.s_read[g - 2] == NWARP, f"S_{g} overwrote S_{g - 2} before every warp read it")
+            self.check(self.pv_exec[g - 2] or not self.keep[g - 2], f"S_{g} overwrote P_{g - 2} before its P.V")
         self.s_exec[g] = True
 
     def _read_s(self, g):
-        self._check(self.s_exec[g], f"softmax read S_{g} before it was computed")
+        self.check(self.s_exec[g], f"softmax read S_{g} before it was computed")
         self.s_read[g] += 1
 
     def _exec_pv(self, g, i, first):
-        self._check(self.p_written[g] == NWARP, f"P.V of tile {g} read an incomplete P")
-        self._check(self.v_slot[g % VST] == g, f"P.V of tile {g} read a V slot holding tile {self.v_slot[g % VST]}")
+        self.check(self.p_written[g] == NWARP, f"P.V of tile {g} read an incomplete P")
+        self.check(self.v_slot[g % VST] == g, f"P.V of tile {g} read a V slot holding tile {self.v_slot[g % VST]}")
         if first and i >= 2:
-            self._check(self.o_read.get(i - 2, 0) == NWARP, f"split {i} overwrote the O of split {i - 2} before it was read")
+            self.check(self.o_read.get(i - 2, 0) == NWARP, f"split {i} overwrote the O of split {i - 2} before it was read")
         self.pv_exec[g] = True
 
     def _check_o_current(self, g, n, what):
         for h, (m, t) in enumerate(self.tiles):
             if m == n and h < g and self.keep[h]:
-                self._check(self.pv_exec[h], f"O {what} at tile {g} before the P.V of tile {h}")
+                self.check(self.pv_exec[h], f"O {what} at tile {g} before the P.V of tile {h}")
 
     def _read_o(self, n, i):
         self._check_o_current(len(self.tiles), n, "read out")
         self.o_read[i] = self.o_read.get(i, 0) + 1
 
-    # ------------------------------------------------------------ scheduler
-    def run(self, max_steps=200000):
-        rng = self.rng
+    def run(self):
         roles = [("producer", self.producer()), ("loader", self.loader()), ("mma", self.mma())]
         roles += [(f"softmax{w}", self.softmax(w)) for w in range(NWARP)]
-        pend = {name: None for name, _ in roles}
-        done = set()
-        nbar_wait = {}
-        speed = {name: rng.uniform(0.05, 1.0) for name, _ in roles}
-        speed["pipe"], speed["tma"] = rng.uniform(0.05, 1.0), rng.uniform(0.05, 1.0)
-        gens = dict(roles)
-        idle = 0
-        for _ in range(max_steps):
-            cands = [n for n in gens if n not in done]
-            if self.queue:
-                cands.append("pipe")
-            if self.tma:
-                cands.append("tma")
-            if not cands:
-                return
-            who = rng.choices(cands, weights=[speed[c] for c in cands])[0]
-            progressed = False
-            if who == "pipe":
-                kind, x = self.queue.pop(0)
-                x() if kind == "op" else x.arrive()
-                progressed = True
-            elif who == "tma":
-                bar, land = self.tma.pop(rng.randrange(len(self.tma)))
-                land()
-                bar.arrive()
-                progressed = True
-            else:
-                if pend[who] is None:
-                    try:
-                        pend[who] = next(gens[who])
-                    except StopIteration:
-                        done.add(who)
-                        continue
-                cmd = pend[who]
-                if cmd[0] == "wait":
-                    bar, k = cmd[1], cmd[2]
-                    if bar.phase >= k + 2:
-                        raise ProtocolError(f"{who} waits for completion {k} of {bar.name}, which is already at {bar.phase}")
-                    if bar.phase == k + 1:
-                        pend[who], progressed = None, True
-                    elif bar.phase % 2 != k % 2:
-                        raise ProtocolError(f"{who} waits for completion {k} of {bar.name} at phase {bar.phase}: early return")
-                elif cmd[0] == "nbar":
-                    if who not in nbar_wait:
-                        nbar_wait[who] = self.nbar_gen
-                        self.nbar_count += 1
-                        if self.nbar_count == NWARP:
-                            self.nbar_gen += 1
-                            self.nbar_count = 0
-                        progressed = True
-                    if nbar_wait[who] < self.nbar_gen:
-                        del nbar_wait[who]
-                        pend[who], progressed = None, True
-                else:
-                    if cmd[0] == "arrive":
-                        cmd[1].arrive()
-                    elif cmd[0] == "tma":
-                        self.tma.append((cmd[1], cmd[2]))
-                    elif cmd[0] in ("op", "commit"):
-                        self.queue.append((cmd[0], cmd[1]))
-                    elif cmd[0] == "do":
-                        cmd[1]()
-                    pend[who], progressed = None, True
-            idle = 0 if progressed else idle + 1
-            if idle > 5000:
-                raise ProtocolError(f"deadlock: {sorted(n for n in gens if n not in done)} blocked on "
-                                    f"{[(n, pend[n][:1], getattr(pend[n][1], 'name', None)) for n in gens if n not in done and pend[n]]}")
-        raise ProtocolError("step limit")
+        Sim.run(self, roles, nbar_size=NWARP)
 
 
 def _random_items(rng):
