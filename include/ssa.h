@@ -199,6 +199,17 @@ int ssa_decode(const void* q, const void* k, const void* v, void* out, float* ls
 /* Bytes of workspace ssa_decode needs for this shape (0 for invalid sizes). */
 size_t ssa_decode_workspace_bytes(int B, int Hq, int Lq, int d, int num_splits);
 
+/* A num_splits for ssa_decode on a GPU with num_sms SMs.  The decode kernel is
+ * persistent: one CTA per SM takes the B * Hkv * num_splits work items
+ * (split, KV head, sequence) round-robin.  Returned: the split count s, at
+ * most 256 and at most nK = ceil(Lk / Bc), that minimises the work of the
+ * busiest CTA, ceil(B * Hkv * s / num_sms) * (ceil(nK / s) + 1) key tiles
+ * (one tile's worth per split for its query rows, partial results and
+ * merge); counts that would leave a split empty are passed over and ties go
+ * to fewer splits.  Host only.  0 for invalid arguments (Bc not 64 or 128,
+ * or a non-positive size). */
+int ssa_decode_default_splits(int B, int Hkv, int Lk, int Bc, int num_sms);
+
 /* Human-readable name of a status code (static storage). */
 const char* ssa_status_string(int status);
 

@@ -618,6 +618,26 @@ size_t ssa_decode_workspace_bytes(int B, int Hq, int Lq, int d, int num_splits) 
   return ssa_dec::workspace_bytes(B, Hq, Lq, d, num_splits);
 }
 
+int ssa_decode_default_splits(int B, int Hkv, int Lk, int Bc, int num_sms) {
+  if (B <= 0 || Hkv <= 0 || Lk <= 0 || (Bc != 64 && Bc != 128) || num_sms <= 0) return 0;
+  const long long pairs = (long long)B * Hkv;
+  const int nK = (int)(((long long)Lk + Bc - 1) / Bc);
+  const int smax = nK < 256 ? nK : 256;
+  int best = 1;
+  long long best_cost = -1;
+  for (int s = 1; s <= smax; ++s) {
+    const int T = (nK + s - 1) / s;  // key tiles per split
+    if ((nK + T - 1) / T < s) continue;  // would leave empty splits: a smaller count does the same
+    const long long rounds = (pairs * s + num_sms - 1) / num_sms;  // items of the busiest CTA
+    const long long cost = rounds * (T + 1);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
 int ssa_decode(const void* q, const void* k, const void* v, void* out, float* lse,
                int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
                float scale, float lambda, int Bc, int num_splits, void* workspace,

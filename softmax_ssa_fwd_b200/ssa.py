@@ -25,7 +25,7 @@ MODE_DENSE, MODE_SKIP, MODE_NM = 0, 1, 2
 
 EXPORTED = ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
             "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version",
-            "ssa_decode", "ssa_decode_workspace_bytes", "ssa_fwd_blockmask"]
+            "ssa_decode", "ssa_decode_workspace_bytes", "ssa_decode_default_splits", "ssa_fwd_blockmask"]
 
 
 class SSAError(RuntimeError):
@@ -62,6 +62,8 @@ def _load():
     lib.ssa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, F, I, I, P, ctypes.c_size_t, P]
     lib.ssa_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.ssa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
+    lib.ssa_decode_default_splits.restype = I
+    lib.ssa_decode_default_splits.argtypes = [I, I, I, I, I]
     return lib
 
 
@@ -164,6 +166,10 @@ def ssa_decode_workspace_bytes(B, Hq, Lq, d, num_splits) -> int:
     return int(lib.ssa_decode_workspace_bytes(B, Hq, Lq, d, num_splits))
 
 
+def ssa_decode_default_splits(B, Hkv, Lk, Bc, num_sms) -> int:
+    return int(lib.ssa_decode_default_splits(B, Hkv, Lk, Bc, num_sms))
+
+
 def ssa_decode(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, lam, Bc,
                num_splits, workspace, workspace_bytes, stream=None) -> int:
     """Direct call of the decode entry point; returns its status code."""
@@ -178,17 +184,17 @@ def decode(q, k, v, *, causal=True, scale=None, lam=0.0, Bc=128, num_splits=None
 
     q [B, Lq, Hq, d] (a few rows), k/v [B, Lk, Hkv, d] bf16 CUDA tensors.  Returns
     (out [B, Lq, Hq, d] bf16, lse [B, Hq, Lq] fp32, tile_skip_count [B, Hq] int32).
-    num_splits defaults to enough key splits for about two work items per SM (the
+    num_splits defaults to ssa_decode_default_splits for this GPU's SM count (the
     kernel is persistent: one CTA per SM takes the (split, KV head, sequence) items in turn).
     """
     B, Lq, Hq, d = q.shape
     _, Lk, Hkv, _ = k.shape
     if scale is None:
         scale = d ** -0.5
-    nK = -(-Lk // Bc)
     if num_splits is None:
         sms = torch.cuda.get_device_properties(q.device).multi_processor_count
-        num_splits = max(1, min(nK, -(-2 * sms // (B * Hkv))))
+        # 0 for arguments ssa_decode rejects: it then reports why
+        num_splits = ssa_decode_default_splits(B, Hkv, Lk, Bc, sms) or 1
     if out is None:
         out = torch.empty_like(q)
     if lse is None:

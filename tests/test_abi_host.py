@@ -30,7 +30,7 @@ def test_header_declares_the_entry_points():
     assert _declared_functions() == sorted(
         ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
          "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version",
-         "ssa_decode", "ssa_decode_workspace_bytes", "ssa_fwd_blockmask"])
+         "ssa_decode", "ssa_decode_workspace_bytes", "ssa_decode_default_splits", "ssa_fwd_blockmask"])
 
 
 def test_library_exports_every_declared_symbol(ssa):
@@ -138,6 +138,40 @@ def test_decode_workspace_bytes(ssa):
     # (max, sum)), then the skip counts per (batch, head, split)
     assert ssa.ssa_decode_workspace_bytes(8, 32, 1, 128, 16) == 8 * 32 * 16 * 4 * (128 * 4 + 8) + 8 * 32 * 16 * 4
     assert ssa.ssa_decode_workspace_bytes(0, 32, 1, 128, 16) == 0
+
+
+def _busiest_cta_tiles(pairs, nK, s, sms):
+    """Key tiles (plus one per split) walked by the busiest CTA when the
+    pairs * s work items are handed to sms CTAs round-robin."""
+    T = -(-nK // s)
+    load = [0] * sms
+    for it in range(pairs * s):
+        sp = it % s
+        nt = max(0, min(nK, (sp + 1) * T) - sp * T)
+        load[it % sms] += nt + (1 if nt else 0)
+    return max(load)
+
+
+@pytest.mark.parametrize("B,Hkv,Lk,Bc,sms", [(8, 8, 32768, 128, 148), (1, 8, 4096, 128, 148),
+                                             (1, 1, 1000, 64, 148), (64, 8, 8192, 128, 148),
+                                             (2, 4, 300000, 128, 132)])
+def test_decode_default_splits_balances_the_persistent_grid(ssa, B, Hkv, Lk, Bc, sms):
+    nK = -(-Lk // Bc)
+    s = ssa.ssa_decode_default_splits(B, Hkv, Lk, Bc, sms)
+    assert 1 <= s <= min(nK, 256)
+    T = -(-nK // s)
+    assert -(-nK // T) == s  # no split is left empty
+    # the busiest CTA, simulated item by item, is within 10 % of the best count's
+    best = min(_busiest_cta_tiles(B * Hkv, nK, c, sms) for c in range(1, min(nK, 256) + 1))
+    assert _busiest_cta_tiles(B * Hkv, nK, s, sms) <= 1.10 * best
+
+
+def test_decode_default_splits_rejects_bad_arguments(ssa):
+    assert ssa.ssa_decode_default_splits(0, 8, 4096, 128, 148) == 0
+    assert ssa.ssa_decode_default_splits(1, 8, 4096, 32, 148) == 0
+    assert ssa.ssa_decode_default_splits(1, 8, 4096, 128, 0) == 0
+    # (sequence, KV head) pairs that fill the GPU evenly: no split
+    assert ssa.ssa_decode_default_splits(37, 8, 4096, 128, 148) == 1
 
 
 def test_blockmask_argument_checks(ssa):
