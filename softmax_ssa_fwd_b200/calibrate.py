@@ -100,6 +100,38 @@ def skip_enabled(step: int, initial_disabled_steps: int) -> bool:
     return step >= initial_disabled_steps
 
 
+def skip_enabled_at_timestep(timestep: float, disabled_until_timestep: float | None) -> bool:
+    """Timestep cutoff of diffusion models ("Refactor Skip Softmax Attention
+    Interface", summary item 5: a normalized-timestep cutoff,
+    ``disabled_until_timestep``).  The page names the knob only; the reading
+    taken: the denoising timestep is normalized to [0, 1] and falls over the
+    run, skip-softmax stays off while it is above the cutoff and is on from the
+    first step at or below it.  ``None`` means no cutoff."""
+    if not 0.0 <= timestep <= 1.0:
+        raise ValueError("timestep must be normalized to [0, 1]")
+    if disabled_until_timestep is None:
+        return True
+    if not 0.0 <= disabled_until_timestep <= 1.0:
+        raise ValueError("disabled_until_timestep must lie in [0, 1]")
+    return timestep <= disabled_until_timestep
+
+
+def skip_phase(step: int, timestep: float | None = None, *, initial_disabled_steps: int = 0,
+               disabled_until_timestep: float | None = None) -> bool:
+    """True when a denoising step runs skip-softmax, False when it runs dense:
+    both gates (step count and timestep cutoff) must let it through.  The phase
+    decides the ``mode`` passed to the kernel, and a CUDA graph captured in one
+    phase replays that phase, so captured graphs are keyed by it (the same page
+    keys graphs by the resolved phase)."""
+    if not skip_enabled(step, initial_disabled_steps):
+        return False
+    if timestep is None:
+        if disabled_until_timestep is not None:
+            raise ValueError("a timestep cutoff needs the step's timestep")
+        return True
+    return skip_enabled_at_timestep(timestep, disabled_until_timestep)
+
+
 def fit_from_sweep(points: Sequence[tuple], seq_k: int) -> dict:
     """Fit (a, b) from sweep output: each lambda becomes a scale factor
     lambda * seq_k at its achieved sparsity; points with zero or full sparsity

@@ -76,3 +76,32 @@ def test_calibrate_hits_its_own_fit():
     fit = calibrate.calibrate(q, k, v, 0.5, scale=w.scale)
     assert fit["a"] > 0 and math.isfinite(fit["b"])
     assert fit["lambda"] == pytest.approx(fit["a"] * math.exp(fit["b"] * 0.5) / w.L)
+
+
+def test_timestep_cutoff_gate():
+    from softmax_ssa_fwd_b200.calibrate import skip_enabled_at_timestep
+    assert skip_enabled_at_timestep(0.9, None)
+    assert not skip_enabled_at_timestep(0.9, 0.5)
+    assert skip_enabled_at_timestep(0.5, 0.5)       # on from the first step at the cutoff
+    assert skip_enabled_at_timestep(0.1, 0.5)
+    # over a run with falling timesteps the gate switches on once and stays on
+    ts = [1.0 - i / 49 for i in range(50)]
+    on = [skip_enabled_at_timestep(t, 0.3) for t in ts]
+    first = on.index(True)
+    assert not any(on[:first]) and all(on[first:]) and ts[first] <= 0.3 < ts[first - 1]
+    for bad in ((1.5, 0.5), (-0.1, 0.5), (0.5, 1.2)):
+        with pytest.raises(ValueError):
+            skip_enabled_at_timestep(*bad)
+
+
+def test_skip_phase_needs_both_gates():
+    from softmax_ssa_fwd_b200.calibrate import skip_phase
+    assert skip_phase(0)
+    assert not skip_phase(2, initial_disabled_steps=3)
+    assert skip_phase(3, initial_disabled_steps=3)
+    assert not skip_phase(10, 0.8, initial_disabled_steps=3, disabled_until_timestep=0.5)
+    assert not skip_phase(1, 0.2, initial_disabled_steps=3, disabled_until_timestep=0.5)
+    assert skip_phase(10, 0.2, initial_disabled_steps=3, disabled_until_timestep=0.5)
+    with pytest.raises(ValueError):
+        skip_phase(10, None, disabled_until_timestep=0.5)
+
