@@ -9,4 +9,5 @@ compiles it (``build()``) and marshals numpy arrays into it (``run_items``).
 """
 from .oracle import build, lib_path, run_items, visited_tiles, OracleResult  # noqa: F401
 # fp64 numpy oracles of the two further paths (same test-infrastructure rule):
-# oracle.decode (split-KV decode) and oracle.blockmask (caller-selected key blocks)
+# oracle.decode (split-KV decode), oracle.blockmask (caller-selected key blocks) and
+# oracle.proxy (selected blocks exact, omitted ones through caller-supplied summaries)
