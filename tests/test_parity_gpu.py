@@ -10,8 +10,7 @@ import pytest
 import torch
 
 from parity_util import all_items, compare, gpu_run
-from softmax_ssa_fwd_b200.inputs import (MODE_DENSE, MODE_NM, MODE_SKIP, WORKLOADS, Workload,
-                                         make_inputs, sample_items)
+from softmax_ssa_fwd_b200.inputs import MODE_DENSE, MODE_NM, MODE_SKIP, WORKLOADS, make_inputs, sample_items
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
