@@ -30,13 +30,15 @@ def block_selected(mask_words, b, hkv, qt, kt) -> bool:
 
 
 def run(q, k, v, mask_words, *, causal: bool, scale: float, lam: float, Br: int, Bc: int,
-        items=None, marginal=None, margin_rel: float = 1e-3):
+        items=None, marginal=None, margin_rel: float = 1e-3, skip_bits=None, marginal_bits=None):
     """q [B, Lq, Hq, d], k/v [B, Lk, Hkv, d]; mask_words [B, Hkv, nQ, ceil(nK/32)] uint32.
 
     Returns (out [B, Lq, Hq, d], lse [B, Hq, Lq], skip_count [B, Hq, nQ], visited [B, Hq, nQ])
     over ``items`` (b, hq, qt) (all by default); other entries stay 0 / -inf.  If
     ``marginal`` (an int array [B, Hq, nQ]) is given it receives, per query tile, the
-    number of visited tiles whose decision lies within margin_rel * lambda of the threshold."""
+    number of visited tiles whose largest row ratio exp(tile_max - running_max) lies within
+    margin_rel * lambda of lambda.  ``skip_bits`` / ``marginal_bits`` (bool arrays
+    [B, Hq, nQ, nK]), if given, receive per key tile the skip decision and that flag."""
     B, Lq, Hq, d = q.shape
     Lk, Hkv = k.shape[1], k.shape[2]
     G = Hq // Hkv
@@ -70,23 +72,28 @@ def run(q, k, v, mask_words, *, causal: bool, scale: float, lam: float, Br: int,
             c0, c1 = kt * Bc, min(Lk, (kt + 1) * Bc)
             st = s[:, c0:c1]
             mt = st.max(axis=1)
-            neg = True
-            near = False
+            # the tile's margin quantity: its largest row ratio exp(mt - m)
+            # (0 for a row with no key here, +inf for a row with no kept key
+            # yet); skipped iff it is below lambda
+            big = 0.0
             for i in range(rows):
                 if mt[i] == -np.inf:
-                    continue
-                if m[i] == -np.inf:
-                    neg = False
-                    continue
-                e = math.exp(mt[i] - m[i])
-                if lam > 0 and abs(e - lam) < margin_rel * lam:
-                    near = True
-                if not (e < lam):
-                    neg = False
-            if near and marginal is not None:
-                marginal[b, hq, qt] += 1
-            if neg:
+                    e = 0.0
+                elif m[i] == -np.inf:
+                    e = math.inf
+                else:
+                    e = math.exp(mt[i] - m[i])
+                big = max(big, e)
+            near = math.isfinite(big) and abs(big - lam) < margin_rel * lam
+            if near:
+                if marginal is not None:
+                    marginal[b, hq, qt] += 1
+                if marginal_bits is not None:
+                    marginal_bits[b, hq, qt, kt] = True
+            if big < lam:
                 skips[b, hq, qt] += 1
+                if skip_bits is not None:
+                    skip_bits[b, hq, qt, kt] = True
                 continue
             mn = np.maximum(m, mt)
             ref = np.where(mn == -np.inf, 0.0, mn)

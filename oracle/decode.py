@@ -34,7 +34,7 @@ class DecodeResult:
     lse: np.ndarray          # [B, Hq, Lq] float64 (natural log)
     skip_count: np.ndarray   # [B, Hq] int64
     skip_bits: np.ndarray    # [B, Hq, nK] bool: tile skipped (by its split)
-    marginal: np.ndarray     # [B, Hq, nK] bool: decision within 1e-3 * lambda of the threshold
+    marginal: np.ndarray     # [B, Hq, nK] bool: the tile's largest row ratio within 1e-3 * lambda of lambda
 
 
 def _as64(t) -> np.ndarray:
@@ -76,20 +76,20 @@ def decode(q, k, v, *, causal: bool, scale: float, lam: float, Bc: int, num_spli
                 c0, c1 = kt * Bc, min(Lk, (kt + 1) * Bc)
                 st = s[:, c0:c1]
                 mt = st.max(axis=1)
-                neg = np.ones(Lq, dtype=bool)
-                near = False
+                # the tile's margin quantity: its largest row ratio exp(mt - m)
+                # (0 for a row with no key here, +inf for a row with no kept
+                # key yet); skipped iff it is below lambda
+                big = 0.0
                 for i in range(Lq):
                     if mt[i] == -np.inf:
-                        continue
-                    if m[i] == -np.inf:
-                        neg[i] = False
-                        continue
-                    e = math.exp(mt[i] - m[i])
-                    neg[i] = e < lam
-                    if lam > 0 and abs(e - lam) < margin_rel * lam:
-                        near = True
-                marginal[b, hq, kt] = near
-                if neg.all():
+                        e = 0.0
+                    elif m[i] == -np.inf:
+                        e = math.inf
+                    else:
+                        e = math.exp(mt[i] - m[i])
+                    big = max(big, e)
+                marginal[b, hq, kt] = math.isfinite(big) and abs(big - lam) < margin_rel * lam
+                if big < lam:
                     skip_count[b, hq] += 1
                     skip_bits[b, hq, kt] = True
                     continue

@@ -34,20 +34,25 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def bind(path: str):
+    """Load a compiled oracle library and declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    D = ctypes.c_double
+    lib.ssa_oracle_items.restype = I
+    lib.ssa_oracle_items.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, D, I, I, I, I, I, I, D,
+                                     P, I, P, P, P, P, P, P, P, P, P, I]
+    lib.ssa_oracle_visited_tiles.restype = I
+    lib.ssa_oracle_visited_tiles.argtypes = [I, I, I, I, I, I]
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
         build()
-        lib = ctypes.CDLL(_LIB)
-        P = ctypes.c_void_p
-        I = ctypes.c_int
-        D = ctypes.c_double
-        lib.ssa_oracle_items.restype = I
-        lib.ssa_oracle_items.argtypes = [P, P, P, I, I, I, I, I, I, I, D, I, D, I, I, I, I, I, I, D,
-                                         P, I, P, P, P, P, P, P, P, P, I]
-        lib.ssa_oracle_visited_tiles.restype = I
-        lib.ssa_oracle_visited_tiles.argtypes = [I, I, I, I, I, I]
-        _lib = lib
+        _lib = bind(_LIB)
     return _lib
 
 
@@ -82,13 +87,17 @@ def _as_u16(t) -> np.ndarray:
 def run_items(q, k, v, *, causal: bool, scale: float, mode: int, lam: float = 0.0, n: int = 0,
               m: int = 0, sink: int = 0, recent: int = 0, Br: int = 128, Bc: int = 128,
               items=None, keep_bits: bool = False, tie_tol: float = 1e-4,
-              nthreads: int | None = None) -> OracleResult:
+              nthreads: int | None = None, lib=None, flip_bits=None) -> OracleResult:
     """Run the oracle on work items (b, hq, qt); all items when ``items`` is None.
 
     q: [B, Lq, Hq, d], k, v: [B, Lk, Hkv, d], bf16 (torch) or their uint16 bits.
     ``scale`` is rounded to fp32 first, the precision the kernel receives it in.
+    ``lib``: a library from ``bind`` to run instead of the built oracle (tests only).
+    ``flip_bits`` [n_items, ceil(nK/32)] uint32: key tiles whose skip decision is
+    to be the other one -- accepted only on tiles inside the tolerance band
+    (marginal), else ValueError.
     """
-    lib = _load()
+    lib = lib if lib is not None else _load()
     qa, ka, va = _as_u16(q), _as_u16(k), _as_u16(v)
     B, Lq, Hq, d = qa.shape
     _, Lk, Hkv, _ = ka.shape
@@ -111,13 +120,18 @@ def run_items(q, k, v, *, causal: bool, scale: float, mode: int, lam: float = 0.
     tb = np.zeros((nit, Br, Lkw), np.uint32) if keep_bits else None
     if nthreads is None:
         nthreads = len(os.sched_getaffinity(0))
+    fb = None
+    if flip_bits is not None:
+        fb = np.ascontiguousarray(np.asarray(flip_bits, dtype=np.uint32).reshape(nit, nKw))
     scale32 = float(np.float32(scale))
     ptr = lambda a: a.ctypes.data if a is not None else None  # noqa: E731
     rc = lib.ssa_oracle_items(ptr(qa), ptr(ka), ptr(va), B, Hq, Hkv, Lq, Lk, d, int(causal),
                               scale32, int(mode), float(lam), int(n), int(m), int(sink),
                               int(recent), Br, Bc, float(tie_tol), ptr(items), nit, ptr(out),
                               ptr(lse), ptr(cnt), ptr(vis), ptr(sb), ptr(mb), ptr(kb), ptr(tb),
-                              int(nthreads))
+                              ptr(fb), int(nthreads))
+    if rc == -2:
+        raise ValueError("flip_bits names a tile whose decision is not marginal")
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (rc={rc})")
     return OracleResult(items, out, lse, cnt, vis, sb, mb, kb, tb)

@@ -68,9 +68,11 @@ typedef struct {
   int32_t *skip_count;  /* [n_items] */
   int32_t *visited;     /* [n_items] */
   uint32_t *skip_bits;  /* [n_items][nKw] or NULL: bit kt = tile kt visited and skipped */
-  uint32_t *marginal_bits; /* [n_items][nKw] or NULL: bit kt = some row within 1e-3*lambda of the threshold */
+  uint32_t *marginal_bits; /* [n_items][nKw] or NULL: bit kt = the tile's largest row ratio within 1e-3*lambda of lambda */
   uint32_t *keep_bits;  /* [n_items][Br][Lkw] or NULL: bit j = key j kept for this row */
   uint32_t *tie_bits;   /* [n_items][Br][Lkw] or NULL: bit j = key j's N:M fate is a near tie */
+  const uint32_t *flip_bits; /* [n_items][nKw] or NULL: bit kt = take the other decision (marginal tiles only) */
+  int bad_flip;         /* set when flip_bits names a tile that is not marginal */
   int next_item;
   pthread_mutex_t lock;
 } job_t;
@@ -84,6 +86,7 @@ static double bf16_to_double(uint16_t h) {
 }
 
 static void set_bit(uint32_t *words, long idx) { words[idx >> 5] |= 1u << (idx & 31); }
+static int get_bit(const uint32_t *words, long idx) { return (words[idx >> 5] >> (idx & 31)) & 1u; }
 
 /* Number of visited key tiles for a query tile (reading R3). */
 static int visited_tiles(int causal, int Lq, int Lk, int Br, int Bc, int qt) {
@@ -216,23 +219,32 @@ static void run_item(const job_t *J, int it) {
         for (int j = 0; j < cols; ++j)
           if (kept[(size_t)r * Bc + j]) set_bit(J->keep_bits, ((long)it * Br + r) * Lkw * 32 + c0 + j);
     }
-    /* skip test (readings R1, R2) */
+    /* skip test (readings R1, R2).  The tile is skipped iff its largest row
+     * ratio exp(tmax - m) is below lambda: that largest ratio is the tile's
+     * margin quantity, and the tile is "marginal" when it lies within
+     * 1e-3 * lambda of lambda (the method statement's tolerance band).  A row
+     * with no key in this tile has ratio 0; a row with no kept key yet and a
+     * key here has ratio +inf (never negligible, never marginal). */
     if (skip_on) {
-      int all_negligible = 1, marginal = 0;
+      int all_negligible = 1;
+      double max_ratio = 0.0;
       for (int r = 0; r < rows; ++r) {
-        int negligible;
-        if (tmax[r] == NEG_INF) {
-          negligible = 1;
-        } else if (m_run[r] == NEG_INF) {
-          negligible = 0;
-        } else {
-          const double ratio = exp(tmax[r] - m_run[r]);
-          negligible = ratio < J->lambda;
-          if (fabs(ratio - J->lambda) < 1e-3 * J->lambda) marginal = 1;
-        }
-        if (!negligible) all_negligible = 0;
+        double ratio;
+        if (tmax[r] == NEG_INF) ratio = 0.0;
+        else if (m_run[r] == NEG_INF) ratio = INFINITY;
+        else ratio = exp(tmax[r] - m_run[r]);
+        if (!(ratio < J->lambda)) all_negligible = 0;
+        if (ratio > max_ratio) max_ratio = ratio;
       }
+      const int marginal = isfinite(max_ratio) && fabs(max_ratio - J->lambda) < 1e-3 * J->lambda;
       if (marginal && J->marginal_bits) set_bit(J->marginal_bits, (long)it * nKw * 32 + kt);
+      /* Inside the tolerance band either decision is accepted; a caller that
+       * compares against a kernel which took the other one asks for it here
+       * (anywhere else the request is an error). */
+      if (J->flip_bits && get_bit(J->flip_bits, (long)it * nKw * 32 + kt)) {
+        if (!marginal) ((job_t *)J)->bad_flip = 1;
+        all_negligible = !all_negligible;
+      }
       if (all_negligible) {
         ++skipped;
         if (J->skip_bits) set_bit(J->skip_bits, (long)it * nKw * 32 + kt);
@@ -285,8 +297,9 @@ static void *worker(void *arg) {
   return NULL;
 }
 
-/* Entry point.  Returns 0, or -1 on an argument it cannot evaluate.  Output
- * bit arrays must be zeroed by the caller.  Work items are independent, so
+/* Entry point.  Returns 0, -1 on an argument it cannot evaluate, or -2 when
+ * flip_bits asks for the other decision on a tile that is not marginal.
+ * Output bit arrays must be zeroed by the caller.  Work items are independent, so
  * they are spread over nthreads threads; each item's arithmetic is serial. */
 int ssa_oracle_items(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int Hq, int Hkv,
                      int Lq, int Lk, int d, int causal, double scale, int mode, double lambda, int n,
@@ -294,7 +307,7 @@ int ssa_oracle_items(const uint16_t *q, const uint16_t *k, const uint16_t *v, in
                      const int32_t *items, int n_items, double *out, double *lse,
                      int32_t *skip_count, int32_t *visited, uint32_t *skip_bits,
                      uint32_t *marginal_bits, uint32_t *keep_bits, uint32_t *tie_bits,
-                     int nthreads) {
+                     const uint32_t *flip_bits, int nthreads) {
   if (!q || !k || !v || !items || !out || !lse || !skip_count || !visited) return -1;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Lq <= 0 || Lk <= 0 || d <= 0 || Br <= 0 || Bc <= 0)
     return -1;
@@ -313,6 +326,7 @@ int ssa_oracle_items(const uint16_t *q, const uint16_t *k, const uint16_t *v, in
   J.items = items; J.n_items = n_items; J.out = out; J.lse = lse;
   J.skip_count = skip_count; J.visited = visited; J.skip_bits = skip_bits;
   J.marginal_bits = marginal_bits; J.keep_bits = keep_bits; J.tie_bits = tie_bits;
+  J.flip_bits = flip_bits;
   pthread_mutex_init(&J.lock, NULL);
   if (nthreads < 1) nthreads = 1;
   if (nthreads > 256) nthreads = 256;
@@ -323,7 +337,7 @@ int ssa_oracle_items(const uint16_t *q, const uint16_t *k, const uint16_t *v, in
   if (started == 0) worker(&J);
   for (int t = 0; t < started; ++t) pthread_join(th[t], NULL);
   pthread_mutex_destroy(&J.lock);
-  return 0;
+  return J.bad_flip ? -2 : 0;
 }
 
 /* Visited key tiles of one query tile, exported so tests can pin reading R3. */

@@ -24,3 +24,14 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """One line per GPU/oracle comparison: what was compared and what the
+    tolerance bands excused (visible in -q logs)."""
+    mod = sys.modules.get("parity_util")
+    if mod is None or not mod.REPORTS:
+        return
+    terminalreporter.write_sep("-", "parity reports")
+    for name, rep in mod.REPORTS:
+        terminalreporter.write_line(f"{name}: {rep.line()}")
