@@ -245,6 +245,127 @@ def pack_bits(bits: np.ndarray) -> np.ndarray:
     return words
 
 
+# Every workload of the method's targets, measured on the same device in the
+# same run as the headline (each its own line in the JSON "configs" object):
+# the literal workloads, the two labelled stress variants that make the skip
+# path run, the decode path and the bitmap-selected path.
+SWEEP = [
+    ("tiny lambda=0", "tiny", 0.0, {}),
+    ("tiny lambda=1e-3", "tiny", 1e-3, {}),
+    ("tiny lambda=1e-2", "tiny", 1e-2, {}),
+    ("llama8k lambda=1e-4", "llama8k", 1e-4, {}),
+    ("llama8k lambda=1e-3", "llama8k", 1e-3, {}),
+    ("llama8k lambda=1e-2", "llama8k", 1e-2, {}),
+    ("llama4k_nm24", "llama4k_nm24", 0.0, {}),
+    ("llama4k_nm48", "llama4k_nm48", 0.0, {}),
+    ("wan lambda=1e-3", "wan", 1e-3, {}),
+    ("qwen32k skip+2:4 lambda=1e-3", "qwen32k", 1e-3, {}),
+    ("stress llama8k sink_coef=12 lambda=1e-3", "llama8k", 1e-3, {"sink_coef": 12.0}),
+    ("stress wan local_alpha=2.5 lambda=1e-3", "wan", 1e-3, {"local_alpha": 2.5}),
+    ("llama8k key blocks by bitmap density 0.25 lambda=1e-3", "llama8k", 1e-3, {"mask_density": 0.25}),
+    ("decode qwen32k_decode lambda=1e-4", "qwen32k_decode", 1e-4, {}),
+]
+
+
+def sweep_configs(dev, stream, target_ms: float = 400.0):
+    """Time every SWEEP entry on this GPU: CUDA events on the launching
+    stream, 2 warm-up launches, then enough launches for ~target_ms (at least
+    3).  Workloads smaller than L2 alternate two input sets."""
+    from softmax_ssa_fwd_b200 import ssa
+    bf16_peak, _, hbm_peak, src = peaks()
+    res = {}
+    for label, name, lam, extra in SWEEP:
+        w = WORKLOADS[name]
+        dens = extra.get("mask_density", 0.0)
+        kw = {k_: v_ for k_, v_ in extra.items() if k_ != "mask_density"}
+        if kw:
+            w = w.with_(**kw)
+        if w.Lq:  # decode
+            nsets = 2
+            ws_bytes = ssa.ssa_decode_workspace_bytes(w.B, w.Hq, w.Lq, w.d, w.splits)
+            sets = []
+            for si in range(nsets):
+                q, k, v = make_inputs(w.with_(seed=w.seed + 1000 * si), dev)
+                sets.append((q, k, v, torch.empty_like(q),
+                             torch.empty(w.B, w.Hq, w.Lq, dtype=torch.float32, device=dev),
+                             torch.empty(w.B, w.Hq, dtype=torch.int32, device=dev),
+                             torch.empty(ws_bytes, dtype=torch.uint8, device=dev)))
+
+            def launch(i):
+                q, k, v, o, l_, c, ws = sets[i % nsets]
+                return ssa.ssa_decode(q, k, v, o, l_, c, w.B, w.Hq, w.Hkv, w.Lq, w.L, w.d, w.causal, w.scale,
+                                      lam, w.Bc, w.splits, ws, ws_bytes, stream)
+        else:
+            in_bytes = 2 * (w.B * w.L * w.Hq * w.d + 2 * w.B * w.L * w.Hkv * w.d)
+            nsets = 2 if in_bytes < 256e6 else 1
+            sets = []
+            for si in range(nsets):
+                q, k, v = make_inputs(w.with_(seed=w.seed + 1000 * si), dev)
+                sets.append((q, k, v, torch.empty_like(q),
+                             torch.empty(w.B, w.Hq, w.L, dtype=torch.float32, device=dev),
+                             torch.empty(w.B, w.Hq, -(-w.L // w.Br), dtype=torch.int32, device=dev)))
+            mask_bits = mask_dev = None
+            if dens > 0:
+                mask_bits = block_mask_bits(w, dens, seed=w.seed)
+                mask_dev = torch.from_numpy(pack_bits(mask_bits).view(np.int32)).to(dev)
+
+            def launch(i):
+                q, k, v, o, l_, c = sets[i % nsets]
+                if mask_dev is not None:
+                    return ssa.ssa_fwd_blockmask(q, k, v, o, l_, c, w.B, w.Hq, w.Hkv, w.L, w.L, w.d, w.causal,
+                                                 w.scale, w.mode, lam, w.n, w.m, w.sink, w.recent, w.Br, w.Bc,
+                                                 mask_dev, stream)
+                return ssa.ssa_fwd(q, k, v, o, l_, c, w.B, w.Hq, w.Hkv, w.L, w.L, w.d, w.causal, w.scale,
+                                   w.mode, lam, w.n, w.m, w.sink, w.recent, w.Br, w.Bc, stream)
+
+        for i in range(2):
+            if launch(i) != 0:
+                raise RuntimeError(f"{label}: launch refused")
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        launch(0)
+        e1.record(stream)
+        e1.synchronize()
+        steps = max(3, min(500, int(target_ms / max(e0.elapsed_time(e1), 1e-3))))
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(steps):
+            launch(i)
+        e1.record(stream)
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        if ssa.ssa_device_status(stream) != 0:
+            raise RuntimeError(f"{label}: device-side timeout")
+        entry = {"workload": workload_name(w, lam), "ms_per_step": ms, "steps": steps}
+        if w.Lq:
+            nK = -(-w.L // w.Bc)
+            skipped = sum(float(s_[5].sum().item()) for s_ in sets) / nsets
+            visited = float(w.B * w.Hq * nK)
+            gbs = decode_alg_bytes(w) / (ms * 1e-3) / 1e9
+            entry.update({"hbm_gbs": gbs, "hbm_frac_of_peak": gbs / hbm_peak,
+                          "dense_equiv_tflops": dense_equiv_flops(w, Lq=w.Lq) / (ms * 1e-3) / 1e12,
+                          "tiles_skipped_frac": skipped / visited,
+                          "tokens_per_s": w.B * w.Lq / (ms * 1e-3)})
+        else:
+            visited = ssa.ssa_visited_tiles(w.causal, w.L, w.L, w.Br, w.Bc) * w.B * w.Hq
+            if mask_bits is not None:
+                visited = int(mask_bits.sum()) * (w.Hq // w.Hkv)
+            skipped = sum(float(s_[5].sum().item()) for s_ in sets) / nsets
+            kept = visited - skipped
+            fd = dense_equiv_flops(w) / (ms * 1e-3) / 1e12
+            fe = 2.0 * w.Br * w.Bc * w.d * (visited + kept) / (ms * 1e-3) / 1e12
+            entry.update({"dense_equiv_tflops": fd, "executed_tflops": fe,
+                          "executed_frac_of_peak": fe / bf16_peak, "dense_equiv_frac_of_peak": fd / bf16_peak,
+                          "tiles_skipped_frac": skipped / visited, "tiles_visited": visited,
+                          "tokens_per_s": w.B * w.L / (ms * 1e-3)})
+        res[label] = entry
+        del sets
+        torch.cuda.empty_cache()
+    res["_peak"] = {"bf16_tflops": bf16_peak, "hbm_gbs": hbm_peak, "source": f"{src} (burst)"}
+    return res
+
+
 def decode_cpu_baseline(w, lam, budget_s: float, seed: int = 7):
     """The fp64 decode oracle (numpy) on a bounded sample of (sequence, head)
     pairs of the decode workload; dense-equivalent FLOPs of the sample / wall."""
@@ -398,6 +519,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--splits", type=int, default=None, help="decode: override the key splits")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload sweep that fills the line's \"configs\" object")
     ap.add_argument("--mask-density", type=float, default=0.0,
                     help="select key blocks by a seeded random bitmap of this density "
                          "(ssa_fwd_blockmask); key tile 0 and the diagonal tile always selected")
@@ -555,6 +678,14 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, lam, args.cpu_budget)
 
+    configs = None
+    if world == 1 and not args.no_configs:
+        del sets
+        torch.cuda.empty_cache()
+        with Clocks(local_rank) as clk_sweep:
+            configs = sweep_configs(dev, stream)
+        configs["_clocks"] = clk_sweep.summary()
+
     if rank == 0:
         clocks = clk.summary()
         line = {
@@ -583,6 +714,7 @@ def main():
             "e2e": e2e,
             "cpu_baseline": cpu,
             "kernel_hash": kernel_hash(),
+            "configs": configs,
         }
         alg_bytes = 2 * (2 * w.B * w.L * w.Hq * w.d + 2 * w.B * w.L * w.Hkv * w.d) + 4 * w.B * w.Hq * w.L
         line["roofline"]["hbm_frac_of_algorithmic_bytes"] = alg_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak

@@ -21,8 +21,9 @@
  *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers on the current CUDA device,
- *     16-byte aligned, contiguous, owned by the caller.  The library keeps no
- *     reference to them after the call returns.
+ *     contiguous, owned by the caller; bf16 and fp32 tensors 16-byte aligned,
+ *     int32 / uint32 arrays 4-byte aligned (SSA_ERR_INVALID_ARG otherwise).
+ *     The library keeps no reference to them after the call returns.
  *   - q:   [B, Lq, Hq, d]  bf16
  *     k,v: [B, Lk, Hkv, d] bf16
  *     out: [B, Lq, Hq, d]  bf16 (overwritten)
@@ -76,7 +77,7 @@ int ssa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
             float scale, int mode, float lambda, int n, int m, int sink, int recent, int Br, int Bc,
             void* stream);
 
-/* Same kernel as ssa_fwd, also writing per-tile evidence (either may be NULL):
+/* Same kernel as ssa_fwd, also writing per-tile evidence (any may be NULL):
  *   skip_bits: [B, Hq, nQ, ceil(nK / 32)] uint32, nK = ceil(Lk / Bc); bit kt of
  *              query tile qt is set iff key tile kt was visited and skipped.
  *              Every word of every query tile is written.
@@ -84,12 +85,19 @@ int ssa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
  *              j is visible to row i and kept by N:M (every visible key when N:M
  *              is off), for the key tiles the row's query tile visits.  Words of
  *              tiles that are not visited are not written: zero the buffer first.
+ *   v_tile_loads: [B, Hq, ceil(nQp / 2)] int32, nQp = ceil(Lq / 128): the
+ *              number of V tiles the CTA that owns query rows
+ *              [256 p, 256 p + 256) of (b, hq) loaded.  The kernel loads V
+ *              tile kt only once one of those rows' query tiles has decided to
+ *              keep key tile kt, so this equals the number of key tiles kept by
+ *              at least one of them (the evidence that a skipped tile never
+ *              issues its V load).
  * Skipped tiles still report their keep bits (the N:M mask precedes the skip). */
 int ssa_fwd_debug(const void* q, const void* k, const void* v, void* out, float* lse,
                   int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d,
                   int causal, float scale, int mode, float lambda, int n, int m, int sink,
                   int recent, int Br, int Bc, void* stream, uint32_t* skip_bits,
-                  uint32_t* keep_bits);
+                  uint32_t* keep_bits, int32_t* v_tile_loads);
 
 /* Allocation-free variant of ssa_fwd (the pages have no counterpart; this is
  * a service of this library).  Same arguments, layouts and results as
@@ -109,8 +117,8 @@ int ssa_fwd_debug(const void* q, const void* k, const void* v, void* out, float*
  * call on a device and keeps the last call's contents: each call clears the
  * status word on `stream` before its kernel starts.  Calls that overlap on the
  * GPU (on different streams) therefore race on that word; serialise them.
- * A timed-out wait still makes the kernel unwind, but this entry point does
- * not report it (ssa_device_status reads ssa_fwd's word, not this one).
+ * A timed-out wait makes the kernel unwind and raise that word;
+ * ssa_device_status (which allocates nothing either) reads and clears it.
  * The first call on a device looks up the array's device address (with that
  * device current); later calls reuse it.
  * Returns SSA_OK once enqueued, or the status codes of ssa_fwd. */
@@ -141,6 +149,17 @@ int ssa_fwd_blockmask(const void* q, const void* k, const void* v, void* out, fl
                       int causal, float scale, int mode, float lambda, int n, int m, int sink,
                       int recent, int Br, int Bc, const uint32_t* block_mask, void* stream);
 
+/* Same kernel as ssa_fwd_blockmask, also writing evidence (either may be NULL):
+ *   skip_bits:    [B, Hq, nQ, ceil(nK / 32)] uint32; bit kt of query tile qt is
+ *                 set iff key tile kt was selected, visible, and skipped.  Bits
+ *                 are OR-ed in: zero the buffer first.
+ *   v_tile_loads: as in ssa_fwd_debug (V tiles loaded per CTA). */
+int ssa_fwd_blockmask_debug(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                            int causal, float scale, int mode, float lambda, int n, int m, int sink,
+                            int recent, int Br, int Bc, const uint32_t* block_mask, void* stream,
+                            uint32_t* skip_bits, int32_t* v_tile_loads);
+
 /* Total key tiles visited by all query tiles of one (batch, head) pair: a pure
  * function of the shape, used to turn skip counts into skip fractions and
  * executed FLOPs.  Returns -1 for invalid sizes. */
@@ -157,8 +176,10 @@ int64_t ssa_visited_tiles(int causal, int Lq, int Lk, int Br, int Bc);
 void ssa_set_wait_timeout_ns(uint64_t ns);
 
 /* Synchronises `stream`, returns SSA_OK or SSA_ERR_TIMEOUT if a kernel on this
- * device recorded a timed-out wait since the last call, and clears the word.
- * Returns SSA_ERR_CUDA if the synchronisation itself fails. */
+ * device recorded a timed-out wait since the last call (in the status word of
+ * the allocating entry points or in that of ssa_fwd_noalloc), and clears the
+ * word.  Allocates nothing.  Returns SSA_ERR_CUDA if the synchronisation
+ * itself fails. */
 int ssa_device_status(void* stream);
 
 /* Decode-phase skip-softmax attention: a few query rows per sequence (Lq,
@@ -195,6 +216,15 @@ int ssa_decode(const void* q, const void* k, const void* v, void* out, float* ls
                int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
                float scale, float lambda, int Bc, int num_splits, void* workspace,
                size_t workspace_bytes, void* stream);
+
+/* Same kernels as ssa_decode, also writing the skip decisions:
+ *   skip_bits: [B, Hq, ceil(nK / 32)] uint32 (non-NULL); bit kt of (b, hq) is
+ *              set iff key tile kt was skipped for query head hq (by the split
+ *              that owns it).  Bits are OR-ed in: zero the buffer first. */
+int ssa_decode_debug(const void* q, const void* k, const void* v, void* out, float* lse,
+                     int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
+                     float scale, float lambda, int Bc, int num_splits, void* workspace,
+                     size_t workspace_bytes, void* stream, uint32_t* skip_bits);
 
 /* Bytes of workspace ssa_decode needs for this shape (0 for invalid sizes). */
 size_t ssa_decode_workspace_bytes(int B, int Hq, int Lq, int d, int num_splits);

@@ -30,7 +30,8 @@ def block_selected(mask_words, b, hkv, qt, kt) -> bool:
 
 
 def run(q, k, v, mask_words, *, causal: bool, scale: float, lam: float, Br: int, Bc: int,
-        items=None, marginal=None, margin_rel: float = 1e-3, skip_bits=None, marginal_bits=None):
+        items=None, marginal=None, margin_rel: float = 1e-3, skip_bits=None, marginal_bits=None,
+        flip=None):
     """q [B, Lq, Hq, d], k/v [B, Lk, Hkv, d]; mask_words [B, Hkv, nQ, ceil(nK/32)] uint32.
 
     Returns (out [B, Lq, Hq, d], lse [B, Hq, Lq], skip_count [B, Hq, nQ], visited [B, Hq, nQ])
@@ -38,7 +39,9 @@ def run(q, k, v, mask_words, *, causal: bool, scale: float, lam: float, Br: int,
     ``marginal`` (an int array [B, Hq, nQ]) is given it receives, per query tile, the
     number of visited tiles whose largest row ratio exp(tile_max - running_max) lies within
     margin_rel * lambda of lambda.  ``skip_bits`` / ``marginal_bits`` (bool arrays
-    [B, Hq, nQ, nK]), if given, receive per key tile the skip decision and that flag."""
+    [B, Hq, nQ, nK]), if given, receive per key tile the skip decision and that flag.
+    ``flip`` (bool [B, Hq, nQ, nK]): key tiles whose decision is to be the other one;
+    accepted only on marginal tiles, else ValueError."""
     B, Lq, Hq, d = q.shape
     Lk, Hkv = k.shape[1], k.shape[2]
     G = Hq // Hkv
@@ -90,7 +93,12 @@ def run(q, k, v, mask_words, *, causal: bool, scale: float, lam: float, Br: int,
                     marginal[b, hq, qt] += 1
                 if marginal_bits is not None:
                     marginal_bits[b, hq, qt, kt] = True
-            if big < lam:
+            skip = big < lam
+            if flip is not None and flip[b, hq, qt, kt]:
+                if not near:
+                    raise ValueError(f"flip of tile {kt} of {(b, hq, qt)}: not marginal")
+                skip = not skip
+            if skip:
                 skips[b, hq, qt] += 1
                 if skip_bits is not None:
                     skip_bits[b, hq, qt, kt] = True

@@ -44,10 +44,13 @@ def _as64(t) -> np.ndarray:
 
 
 def decode(q, k, v, *, causal: bool, scale: float, lam: float, Bc: int, num_splits: int,
-           heads=None, margin_rel: float = 1e-3) -> DecodeResult:
+           heads=None, margin_rel: float = 1e-3, flip=None) -> DecodeResult:
     """q [B, Lq, Hq, d], k/v [B, Lk, Hkv, d] (torch or numpy, bf16 values).
 
-    ``heads``: optional list of (b, hq) to evaluate (others are left 0 / -inf)."""
+    ``heads``: optional list of (b, hq) to evaluate (others are left 0 / -inf).
+    ``flip``: optional bool [B, Hq, nK]: key tiles whose skip decision is to be
+    the other one; accepted only on marginal tiles (inside the tolerance band),
+    else ValueError."""
     B, Lq, Hq, d = q.shape
     Lk, Hkv = k.shape[1], k.shape[2]
     G = Hq // Hkv
@@ -89,7 +92,12 @@ def decode(q, k, v, *, causal: bool, scale: float, lam: float, Bc: int, num_spli
                         e = math.exp(mt[i] - m[i])
                     big = max(big, e)
                 marginal[b, hq, kt] = math.isfinite(big) and abs(big - lam) < margin_rel * lam
-                if big < lam:
+                skip = big < lam
+                if flip is not None and flip[b, hq, kt]:
+                    if not marginal[b, hq, kt]:
+                        raise ValueError(f"flip of tile {kt} of {(b, hq)}: not marginal")
+                    skip = not skip
+                if skip:
                     skip_count[b, hq] += 1
                     skip_bits[b, hq, kt] = True
                     continue

@@ -85,6 +85,7 @@ struct Params {
   float* o_part;    // [B, Hq, Lq, S * NPART, d]
   float* ml_part;   // [B, Hq, Lq, S * NPART, 2]: running max (log2 units), row sum
   int32_t* sk_part; // [B, Hq, S]
+  uint32_t* skip_bits;  // optional [B, Hq, ceil(nK / 32)]: key tiles skipped (evidence output)
   int* status;
   unsigned long long wait_ns;
   int B, Hq, Hkv, Lq, Lk, causal, S, nK, tiles_per_split, G, R;
@@ -403,7 +404,14 @@ __global__ void __launch_bounds__(NT, 1)
         // lane g < G holds head g's decision; every row reads its own head's
         const bool head_keeps = lane < G && (negs & head_mask) != head_mask;
         const uint32_t keeps = __ballot_sync(0xffffffffu, head_keeps);
-        if (lane < G && !head_keeps) ++skipped;
+        if (lane < G && !head_keeps) {
+          ++skipped;
+          if (p.skip_bits != nullptr && qd == 0) {
+            const int kt = w.kt0 + t;
+            atomicOr(p.skip_bits + ((size_t)w.b * p.Hq + w.hkv * G + lane) * ((p.nK + 31) / 32) + (kt >> 5),
+                     1u << (kt & 31));
+          }
+        }
         const bool mine = valid && ((keeps >> g) & 1u);
         if (keeps != 0u) {
           const float m_new = fmaxf(m_true, mt);
@@ -638,12 +646,15 @@ int ssa_decode_default_splits(int B, int Hkv, int Lk, int Bc, int num_sms) {
   return best;
 }
 
-int ssa_decode(const void* q, const void* k, const void* v, void* out, float* lse,
-               int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
-               float scale, float lambda, int Bc, int num_splits, void* workspace,
-               size_t workspace_bytes, void* stream) {
+static int decode_run(const void* q, const void* k, const void* v, void* out, float* lse,
+                      int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
+                      float scale, float lambda, int Bc, int num_splits, void* workspace,
+                      size_t workspace_bytes, void* stream, uint32_t* skip_bits) {
   using namespace ssa_dec;
   if (!q || !k || !v || !out || !lse || !tile_skip_count || !workspace) return SSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(tile_skip_count) | reinterpret_cast<uintptr_t>(skip_bits) |
+       reinterpret_cast<uintptr_t>(lse)) & 3u)
+    return SSA_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Lk <= 0 || d <= 0 || num_splits <= 0)
     return SSA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return SSA_ERR_INVALID_ARG;
@@ -664,6 +675,7 @@ int ssa_decode(const void* q, const void* k, const void* v, void* out, float* ls
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.skip_count = tile_skip_count;
+  p.skip_bits = skip_bits;
   const size_t rows = (size_t)B * Hq * Lq;
   p.o_part = static_cast<float*>(workspace);
   p.ml_part = p.o_part + rows * num_splits * NPART * d;
@@ -695,6 +707,23 @@ int ssa_decode(const void* q, const void* k, const void* v, void* out, float* ls
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 128) return Bc == 128 ? launch_bc<128, 128>(mk, mv, p, st) : launch_bc<128, 64>(mk, mv, p, st);
   return Bc == 128 ? launch_bc<64, 128>(mk, mv, p, st) : launch_bc<64, 64>(mk, mv, p, st);
+}
+
+int ssa_decode(const void* q, const void* k, const void* v, void* out, float* lse,
+               int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
+               float scale, float lambda, int Bc, int num_splits, void* workspace,
+               size_t workspace_bytes, void* stream) {
+  return decode_run(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, lambda,
+                    Bc, num_splits, workspace, workspace_bytes, stream, nullptr);
+}
+
+int ssa_decode_debug(const void* q, const void* k, const void* v, void* out, float* lse,
+                     int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
+                     float scale, float lambda, int Bc, int num_splits, void* workspace,
+                     size_t workspace_bytes, void* stream, uint32_t* skip_bits) {
+  if (!skip_bits) return SSA_ERR_INVALID_ARG;
+  return decode_run(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, lambda,
+                    Bc, num_splits, workspace, workspace_bytes, stream, skip_bits);
 }
 
 }  // extern "C"

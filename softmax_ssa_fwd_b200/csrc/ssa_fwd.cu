@@ -68,6 +68,7 @@ struct Params {
   int32_t* skip_count;
   uint32_t* skip_bits;  // optional
   uint32_t* keep_bits;  // optional
+  int32_t* v_loads;     // optional [B, Hq, nPairs]: V tile loads each CTA issued
   int* status;
   int B, Hq, Hkv, Lq, Lk, causal, mode, n, m, sink, recent;
   int half;   // Br == 64
@@ -322,9 +323,6 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
   constexpr bool DBG = VAR == 1, MASK = VAR == 2;
   const int nvis = nsteps;  // = max(nvis_h0, nvis_h1) unless key blocks are selected by bitmap
   const bool vote_on = skip_on || MASK;
-  // speculative exponentials are exact only while a skipped tile cannot raise the max
-  const bool spec_ok = p.log2_lambda <= 0.f;
-  bool prev_keep = true;
 
   float m_true = -INFINITY;  // running max over kept tiles (raw q.k units)
   float m_ref = -INFINITY;   // reference the O accumulator and l are scaled to
@@ -434,38 +432,33 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     // the tile", and arrives on the tile's vote barrier for this step's
     // parity.  The MMA warp and the V producer read the same four bytes.
     const uint32_t vbar = smem_u32(&bars->vote_bar[t][j & 1]);
+    bool wkeep = my_vis;
     if (vote_on) {
-      const bool wkeep = (skip_on ? !__all_sync(0xffffffffu, negligible) : true) && my_vis;
+      wkeep = (skip_on ? !__all_sync(0xffffffffu, negligible) : true) && my_vis;
       if (lane == 0) {
         st_shared_u8(smem_u32(&bars->vote[t][j & 1]) + quarter, wkeep ? 1u : 0u);
         mbar_arrive(vbar);
       }
     }
+    // keep_h[h]: logical query tile (half) h keeps this key tile
     bool keep_h[2] = {vis0, vis1};
     // (warp-uniform outcome: the tcgen05 accesses that follow are warp-collective)
-    auto decide = [&]() {
-      if (!__all_sync(0xffffffffu, mbar_wait(vbar, (j >> 1) & 1, p.wait_ns))) {
+    if (vote_on) {
+      if (wkeep) {
+        // A warp with a row that keeps the tile knows that its query tile
+        // keeps it (the tile is skipped only if every row is negligible), so
+        // it goes on at once; the other half's decision does not concern it.
+        keep_h[0] = keep_h[1] = true;
+      } else if (!__all_sync(0xffffffffu, mbar_wait(vbar, (j >> 1) & 1, p.wait_ns))) {
+        // only a warp whose rows are all negligible waits for the others' votes
         if (!failed && lane == 0) record_failure(p, bars);
-        failed = true;
-        return;  // keep the tile
+        failed = true;  // and keeps the tile
+      } else {
+        const uint32_t w = ld_shared_u32(smem_u32(&bars->vote[t][j & 1]));
+        keep_h[0] = p.half ? (w & 0xffffu) != 0u : w != 0u;
+        keep_h[1] = p.half ? (w >> 16) != 0u : w != 0u;
       }
-      const uint32_t w = ld_shared_u32(smem_u32(&bars->vote[t][j & 1]));
-      keep_h[0] = p.half ? (w & 0xffffu) != 0u : w != 0u;
-      keep_h[1] = p.half ? (w >> 16) != 0u : w != 0u;
-    };
-    // With lambda <= 1 a tile that ends up skipped has every row's max below
-    // the running max, so computing its P against the updated max changes
-    // nothing: the exponentials may start before the vote completes.  A
-    // tile right after a skipped one waits for the vote instead, so long
-    // runs of skipped tiles spend no MUFU time.
-    // P of every row for this key tile
-    auto store_zero_p = [&]() {
-      uint32_t pk[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) pk[i] = 0u;
-#pragma unroll
-      for (int h = 0; h < BC / 64; ++h) tmem_st32(lane_base + s_col + 32 * h, pk);
-    };
+    }
     // "P of the first 64 keys is in TMEM" (one arrival per warp, every step)
     auto send_first_half = [&]() {
       tmem_wait_st();
@@ -473,12 +466,8 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->p_half[t]));
     };
-    bool decided = !vote_on;
-    if (!decided && !(spec_ok && prev_keep)) {
-      decide();
-      decided = true;
-    }
-    if (!decided || (half ? keep_h[1] : keep_h[0])) {
+    const bool mine = half ? keep_h[1] : keep_h[0];
+    if (mine) {
       const float m_new = fmaxf(m_true, m_tile);
       bool resc = false;
       float m_ref_new = m_ref, alpha = 1.f;
@@ -509,53 +498,53 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
         }
         tmem_st32(lane_base + s_col + 32 * bb, pk);
       };
-      // the first 64 keys' P, then the decision; the MMA warp may start the
-      // P.V on those keys while the rest of P is computed
+      // the first 64 keys' P; the MMA warp may start the P.V on those keys
+      // while the rest of P is computed
       p_block(0);
-      if (!decided) decide();
-      const bool mine = half ? keep_h[1] : keep_h[0];
-      if (mine) {
-        if (any_resc && n_pv > 0) {
-          // O must be final before this tile's P.V starts (every earlier P.V
-          // of this tile completed before S(j) did)
+      if (any_resc && n_pv > 0) {
+        // O must be final before this tile's P.V starts (every earlier P.V
+        // of this tile completed before S(j) did)
 #pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + o_col + 32 * cc, o);
-            tmem_wait_ld();
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + o_col + 32 * cc, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(lane_base + o_col + 32 * cc, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(lane_base + o_col + 32 * cc, o);
         }
-      } else if (keep_h[0] || keep_h[1]) {
-        // speculated, and only the other half of a 64-row pair keeps it
-        tmem_wait_st();
-        store_zero_p();
       }
       send_first_half();
-      if (mine) {
 #pragma unroll
-        for (int bb = 1; bb < BC / 64; ++bb) p_block(bb);
-        float ls0, ls1;
-        f2_unpack(ls2, ls0, ls1);
-        l = l * alpha + (ls0 + ls1);
-        m_true = m_new;
-        m_ref = m_ref_new;
-      }
+      for (int bb = 1; bb < BC / 64; ++bb) p_block(bb);
+      float ls0, ls1;
+      f2_unpack(ls2, ls0, ls1);
+      l = l * alpha + (ls0 + ls1);
+      m_true = m_new;
+      m_ref = m_ref_new;
     } else {
-      // decided: the tile is skipped, or only the other half of a 64-row
-      // pair keeps it
-      if (keep_h[0] || keep_h[1]) store_zero_p();
+      // the tile is skipped by this query tile; when the other half of a
+      // 64-row pair keeps it, this half's P is zero
+      if (keep_h[0] || keep_h[1]) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pk[i] = 0u;
+#pragma unroll
+        for (int h = 0; h < BC / 64; ++h) tmem_st32(lane_base + s_col + 32 * h, pk);
+      }
       send_first_half();
     }
     const bool tile_keep = keep_h[0] || keep_h[1];
-    const bool my_keep = half ? keep_h[1] : keep_h[0];
-    prev_keep = tile_keep;
+    const bool my_keep = mine;
     if (leader && my_vis) {
       if (!my_keep) {
         ++skipped;
         skip_word |= 1u << (j & 31);
+        if (MASK && p.skip_bits != nullptr) {
+          // steps walk the listed key tiles: record key tile kt itself
+          const int qt = p.half ? 2 * pt + half : pt;
+          atomicOr(p.skip_bits + ((size_t)(b * p.Hq + hq) * p.nQ + qt) * p.nKw + (kt >> 5), 1u << (kt & 31));
+        }
       }
       if (DBG && p.skip_bits != nullptr && ((j & 31) == 31 || j == my_nvis - 1)) {
         const int qt = p.half ? 2 * pt + half : pt;
@@ -786,6 +775,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ======================= V producer =======================
       int last_load[VST];
       for (int i = 0; i < VST; ++i) last_load[i] = -1;
+      int n_loads = 0;  // V tiles this CTA loaded (evidence output)
       for (int j = 0; j < nvis; ++j) {
         if (aborted(bars)) break;
         const int slot = j % VST;
@@ -813,6 +803,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               tma_load_4d(v_s + slot * L::V_BYTES + c * BC * 128, &tm_v, fb, c * 64, wk.hkv, key_tile(j) * BC, wk.b);
             last_load[slot] = j;
             loaded = true;
+            ++n_loads;
           }
         }
         if (fail) {
@@ -831,6 +822,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (last_load[i] >= 0 &&
             !mbar_wait(smem_u32(&bars->v_full[i]), (last_load[i] / VST) & 1, DRAIN_TIMEOUT_NS))
           record_failure(p, bars);
+      if (p.v_loads != nullptr)
+        p.v_loads[((size_t)wk.b * p.Hq + wk.hq) * ((p.nQp + 1) / 2) + wk.pt[0] / 2] = n_loads;
     } else if (warp == 1 && lane == 0 && nvis > 0) {
       // ======================= MMA issuer =======================
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BC, false, false);
@@ -1028,7 +1021,7 @@ template <int D, int BC, int NM_M>
 static int launch_var(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const Params& p, int grid, cudaStream_t stream, int dev, int inst) {
   if (p.block_mask != nullptr) return launch_one<D, BC, NM_M, 2>(mq, mk, mv, p, grid, stream, dev, inst + 2);
-  if (p.skip_bits != nullptr || p.keep_bits != nullptr)
+  if (p.skip_bits != nullptr || p.keep_bits != nullptr || p.v_loads != nullptr)
     return launch_one<D, BC, NM_M, 1>(mq, mk, mv, p, grid, stream, dev, inst + 1);
   return launch_one<D, BC, NM_M, 0>(mq, mk, mv, p, grid, stream, dev, inst);
 }
@@ -1044,12 +1037,14 @@ static int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMa
 }
 
 static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+static bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
 
 static int run(const void* q, const void* k, const void* v, void* out, float* lse,
                int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d, int causal,
                float scale, int mode, float lambda, int n, int m, int sink, int recent, int Br,
                int Bc, void* stream, uint32_t* skip_bits, uint32_t* keep_bits,
-               int* status_override = nullptr, const uint32_t* block_mask = nullptr) {
+               int* status_override = nullptr, const uint32_t* block_mask = nullptr,
+               int32_t* v_loads = nullptr) {
   // ---- argument checks (synchronous, nothing launched on failure)
   if (!q || !k || !v || !out || !lse || !tile_skip_count) return SSA_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Lk <= 0 || d <= 0) return SSA_ERR_INVALID_ARG;
@@ -1059,6 +1054,9 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
   if ((mode & SSA_MODE_SKIP) && (!std::isfinite(lambda) || lambda < 0.f)) return SSA_ERR_INVALID_ARG;
   if ((mode & SSA_MODE_NM) && (sink < 0 || recent < 0)) return SSA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return SSA_ERR_INVALID_ARG;
+  // 32-bit outputs: a misaligned one would fault in the kernel
+  if (!aligned4(tile_skip_count) || !aligned4(skip_bits) || !aligned4(keep_bits) || !aligned4(v_loads))
     return SSA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return SSA_ERR_UNSUPPORTED;
   if ((Br != 64 && Br != 128) || (Bc != 64 && Bc != 128)) return SSA_ERR_UNSUPPORTED;
@@ -1093,6 +1091,7 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
   p.skip_count = tile_skip_count;
   p.skip_bits = skip_bits;
   p.keep_bits = keep_bits;
+  p.v_loads = v_loads;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.Lk = Lk; p.causal = causal ? 1 : 0;
   p.mode = mode;
   p.n = (mode & SSA_MODE_NM) ? n : 0;
@@ -1183,9 +1182,10 @@ int ssa_fwd_debug(const void* q, const void* k, const void* v, void* out, float*
                   int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d,
                   int causal, float scale, int mode, float lambda, int n, int m, int sink,
                   int recent, int Br, int Bc, void* stream, uint32_t* skip_bits,
-                  uint32_t* keep_bits) {
+                  uint32_t* keep_bits, int32_t* v_tile_loads) {
   return ssa::run(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
-                  lambda, n, m, sink, recent, Br, Bc, stream, skip_bits, keep_bits);
+                  lambda, n, m, sink, recent, Br, Bc, stream, skip_bits, keep_bits, nullptr, nullptr,
+                  v_tile_loads);
 }
 
 int ssa_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
@@ -1203,6 +1203,17 @@ int ssa_fwd_blockmask(const void* q, const void* k, const void* v, void* out, fl
   if (!block_mask) return SSA_ERR_INVALID_ARG;
   return ssa::run(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
                   lambda, n, m, sink, recent, Br, Bc, stream, nullptr, nullptr, nullptr, block_mask);
+}
+
+int ssa_fwd_blockmask_debug(const void* q, const void* k, const void* v, void* out, float* lse,
+                            int32_t* tile_skip_count, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                            int causal, float scale, int mode, float lambda, int n, int m, int sink,
+                            int recent, int Br, int Bc, const uint32_t* block_mask, void* stream,
+                            uint32_t* skip_bits, int32_t* v_tile_loads) {
+  if (!block_mask) return SSA_ERR_INVALID_ARG;
+  return ssa::run(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
+                  lambda, n, m, sink, recent, Br, Bc, stream, skip_bits, nullptr, nullptr, block_mask,
+                  v_tile_loads);
 }
 
 int64_t ssa_visited_tiles(int causal, int Lq, int Lk, int Br, int Bc) {
@@ -1223,19 +1234,27 @@ int ssa_device_status(void* stream) {
     return SSA_ERR_CUDA;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= ssa::MAX_DEV) return SSA_ERR_CUDA;
-  int* w;
+  // The two words a timed-out wait can raise on this device: the one the
+  // allocating entry points created (if any has run here) and the static one
+  // of the allocation-free entry point (if it has run here).  Nothing is
+  // allocated: a word that does not exist yet has recorded nothing.
+  int* words[2];
   {
     std::lock_guard<std::mutex> g(ssa::g_mu);
-    w = ssa::status_word(dev);
+    words[0] = ssa::g_status[dev];
+    words[1] = ssa::g_noalloc_addr[dev];
   }
-  if (!w) return SSA_ERR_CUDA;
-  int h = 0;
-  if (cudaMemcpy(&h, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SSA_ERR_CUDA;
-  if (h != 0) {
-    if (cudaMemset(w, 0, sizeof(int)) != cudaSuccess) return SSA_ERR_CUDA;
-    return SSA_ERR_TIMEOUT;
+  bool timed_out = false;
+  for (int* w : words) {
+    if (!w) continue;
+    int h = 0;
+    if (cudaMemcpy(&h, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SSA_ERR_CUDA;
+    if (h != 0) {
+      if (cudaMemset(w, 0, sizeof(int)) != cudaSuccess) return SSA_ERR_CUDA;
+      timed_out = true;
+    }
   }
-  return SSA_OK;
+  return timed_out ? SSA_ERR_TIMEOUT : SSA_OK;
 }
 
 const char* ssa_status_string(int status) {

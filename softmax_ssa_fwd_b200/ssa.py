@@ -25,7 +25,8 @@ MODE_DENSE, MODE_SKIP, MODE_NM = 0, 1, 2
 
 EXPORTED = ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
             "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version",
-            "ssa_decode", "ssa_decode_workspace_bytes", "ssa_decode_default_splits", "ssa_fwd_blockmask"]
+            "ssa_decode", "ssa_decode_debug", "ssa_decode_workspace_bytes", "ssa_decode_default_splits",
+            "ssa_fwd_blockmask", "ssa_fwd_blockmask_debug"]
 
 
 class SSAError(RuntimeError):
@@ -43,7 +44,7 @@ def _load():
     lib.ssa_fwd.restype = I
     lib.ssa_fwd.argtypes = fwd_args
     lib.ssa_fwd_debug.restype = I
-    lib.ssa_fwd_debug.argtypes = fwd_args + [P, P]
+    lib.ssa_fwd_debug.argtypes = fwd_args + [P, P, P]
     lib.ssa_fwd_noalloc.restype = I
     lib.ssa_fwd_noalloc.argtypes = fwd_args
     lib.ssa_visited_tiles.restype = ctypes.c_int64
@@ -58,8 +59,12 @@ def _load():
     lib.ssa_version.argtypes = []
     lib.ssa_fwd_blockmask.restype = I
     lib.ssa_fwd_blockmask.argtypes = fwd_args[:-1] + [P, P]
+    lib.ssa_fwd_blockmask_debug.restype = I
+    lib.ssa_fwd_blockmask_debug.argtypes = fwd_args[:-1] + [P, P, P, P]
     lib.ssa_decode.restype = I
     lib.ssa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, F, I, I, P, ctypes.c_size_t, P]
+    lib.ssa_decode_debug.restype = I
+    lib.ssa_decode_debug.argtypes = lib.ssa_decode.argtypes + [P]
     lib.ssa_decode_workspace_bytes.restype = ctypes.c_size_t
     lib.ssa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.ssa_decode_default_splits.restype = I
@@ -125,16 +130,17 @@ def ssa_fwd_noalloc(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, c
 
 
 def ssa_fwd_debug(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
-                  lam, n, m, sink, recent, Br, Bc, stream=None, skip_bits=None, keep_bits=None) -> int:
+                  lam, n, m, sink, recent, Br, Bc, stream=None, skip_bits=None, keep_bits=None,
+                  v_tile_loads=None) -> int:
     return lib.ssa_fwd_debug(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(tile_skip_count),
                              B, Hq, Hkv, Lq, Lk, d, int(causal), float(scale), int(mode), float(lam),
                              int(n), int(m), int(sink), int(recent), Br, Bc, _stream(stream),
-                             _ptr(skip_bits), _ptr(keep_bits))
+                             _ptr(skip_bits), _ptr(keep_bits), _ptr(v_tile_loads))
 
 
 def attention(q, k, v, *, causal=True, scale=None, mode=MODE_SKIP, lam=0.0, n=0, m=0, sink=0,
               recent=0, Br=128, Bc=128, stream=None, out=None, lse=None, counts=None,
-              skip_bits=None, keep_bits=None):
+              skip_bits=None, keep_bits=None, v_tile_loads=None):
     """Allocate outputs (torch) and run the forward through the C ABI.
 
     q [B, Lq, Hq, d], k/v [B, Lk, Hkv, d] bf16 CUDA tensors.  Returns
@@ -151,12 +157,12 @@ def attention(q, k, v, *, causal=True, scale=None, mode=MODE_SKIP, lam=0.0, n=0,
         lse = torch.empty(B, Hq, Lq, dtype=torch.float32, device=q.device)
     if counts is None:
         counts = torch.empty(B, Hq, nQ, dtype=torch.int32, device=q.device)
-    if skip_bits is None and keep_bits is None:
+    if skip_bits is None and keep_bits is None and v_tile_loads is None:
         st = ssa_fwd(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode, lam,
                      n, m, sink, recent, Br, Bc, stream)
     else:
         st = ssa_fwd_debug(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
-                           lam, n, m, sink, recent, Br, Bc, stream, skip_bits, keep_bits)
+                           lam, n, m, sink, recent, Br, Bc, stream, skip_bits, keep_bits, v_tile_loads)
     if st != SSA_OK:
         raise SSAError(st, "ssa_fwd")
     return out, lse, counts
@@ -178,8 +184,16 @@ def ssa_decode(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal
                           num_splits, _ptr(workspace), int(workspace_bytes), _stream(stream))
 
 
+def ssa_decode_debug(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, lam, Bc,
+                     num_splits, workspace, workspace_bytes, stream=None, skip_bits=None) -> int:
+    return lib.ssa_decode_debug(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(tile_skip_count),
+                                B, Hq, Hkv, Lq, Lk, d, int(causal), float(scale), float(lam), Bc,
+                                num_splits, _ptr(workspace), int(workspace_bytes), _stream(stream),
+                                _ptr(skip_bits))
+
+
 def decode(q, k, v, *, causal=True, scale=None, lam=0.0, Bc=128, num_splits=None, stream=None,
-           out=None, lse=None, counts=None, workspace=None):
+           out=None, lse=None, counts=None, workspace=None, skip_bits=None):
     """Decode-phase skip-softmax attention through the C ABI (torch allocates).
 
     q [B, Lq, Hq, d] (a few rows), k/v [B, Lk, Hkv, d] bf16 CUDA tensors.  Returns
@@ -204,8 +218,13 @@ def decode(q, k, v, *, causal=True, scale=None, lam=0.0, Bc=128, num_splits=None
     nbytes = ssa_decode_workspace_bytes(B, Hq, Lq, d, num_splits)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
-    st = ssa_decode(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale, lam, Bc,
-                    num_splits, workspace, workspace.numel() * workspace.element_size(), stream)
+    nws = workspace.numel() * workspace.element_size()
+    if skip_bits is None:
+        st = ssa_decode(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale, lam, Bc,
+                        num_splits, workspace, nws, stream)
+    else:  # [B, Hq, ceil(nK / 32)], zeroed by the caller
+        st = ssa_decode_debug(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale, lam, Bc,
+                              num_splits, workspace, nws, stream, skip_bits)
     if st != SSA_OK:
         raise SSAError(st, "ssa_decode")
     return out, lse, counts
@@ -220,8 +239,19 @@ def ssa_fwd_blockmask(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d,
                                  int(recent), Br, Bc, _ptr(block_mask), _stream(stream))
 
 
+def ssa_fwd_blockmask_debug(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale,
+                            mode, lam, n, m, sink, recent, Br, Bc, block_mask, stream=None, skip_bits=None,
+                            v_tile_loads=None) -> int:
+    return lib.ssa_fwd_blockmask_debug(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                       _ptr(tile_skip_count), B, Hq, Hkv, Lq, Lk, d, int(causal),
+                                       float(scale), int(mode), float(lam), int(n), int(m), int(sink),
+                                       int(recent), Br, Bc, _ptr(block_mask), _stream(stream),
+                                       _ptr(skip_bits), _ptr(v_tile_loads))
+
+
 def attention_blockmask(q, k, v, block_mask, *, causal=True, scale=None, mode=MODE_SKIP, lam=0.0,
-                        n=0, m=0, sink=0, recent=0, Br=128, Bc=128, stream=None):
+                        n=0, m=0, sink=0, recent=0, Br=128, Bc=128, stream=None, skip_bits=None,
+                        v_tile_loads=None):
     """Forward over the key blocks selected by ``block_mask`` ([B, Hkv, nQ, ceil(nK/32)]
     int32/uint32 CUDA tensor).  Returns (out, lse, tile_skip_count) like ``attention``."""
     B, Lq, Hq, d = q.shape
@@ -232,8 +262,13 @@ def attention_blockmask(q, k, v, block_mask, *, causal=True, scale=None, mode=MO
     out = torch.empty_like(q)
     lse = torch.empty(B, Hq, Lq, dtype=torch.float32, device=q.device)
     counts = torch.empty(B, Hq, nQ, dtype=torch.int32, device=q.device)
-    st = ssa_fwd_blockmask(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode, lam,
-                           n, m, sink, recent, Br, Bc, block_mask, stream)
+    if skip_bits is None and v_tile_loads is None:
+        st = ssa_fwd_blockmask(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
+                               lam, n, m, sink, recent, Br, Bc, block_mask, stream)
+    else:  # skip_bits [B, Hq, nQ, ceil(nK / 32)] zeroed by the caller
+        st = ssa_fwd_blockmask_debug(q, k, v, out, lse, counts, B, Hq, Hkv, Lq, Lk, d, causal, scale,
+                                     mode, lam, n, m, sink, recent, Br, Bc, block_mask, stream,
+                                     skip_bits, v_tile_loads)
     if st != SSA_OK:
         raise SSAError(st, "ssa_fwd_blockmask")
     return out, lse, counts

@@ -30,8 +30,11 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
     """One line per GPU/oracle comparison: what was compared and what the
     tolerance bands excused (visible in -q logs)."""
     mod = sys.modules.get("parity_util")
-    if mod is None or not mod.REPORTS:
+    if mod is None or not (mod.REPORTS or mod.V_LOADS):
         return
     terminalreporter.write_sep("-", "parity reports")
     for name, rep in mod.REPORTS:
         terminalreporter.write_line(f"{name}: {rep.line()}")
+    for name, loaded, walked in mod.V_LOADS:
+        terminalreporter.write_line(f"{name}: V tiles loaded {loaded} of {walked} walked "
+                                    f"({walked - loaded} skipped by every query tile of their CTA)")

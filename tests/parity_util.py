@@ -27,6 +27,7 @@ TIE_TOL = 1e-4
 MARGINAL_FRAC_MAX = 5e-3   # differing decisions inside the band, per visited tile
 TIE_FRAC_MAX = 1e-4        # differing keep bits at near ties, per compared keep bit
 REPORTS = []               # (test id, Report) of every compare(); the terminal summary prints them
+V_LOADS = []               # (test id, V tiles loaded, key tiles walked) of every gpu_run()
 
 
 @dataclass
@@ -53,18 +54,59 @@ class Report:
                 f"lse max-abs {self.lse_max_abs:.2e}")
 
 
+def expected_v_loads(sb_words, causal, Lq, Lk, Br, Bc, selected=None):
+    """V tiles each CTA of the prefill kernel must load, from the kernel's own
+    skip bits (which compare() checks against the oracle): the key tiles that
+    at least one of the CTA's query tiles visits and keeps.  A CTA owns query
+    rows [256 p, 256 p + 256) of one (batch, head): two 128-row query tiles, or
+    four 64-row ones.  ``selected``: bool [B, Hq, nQ, nK] key blocks chosen by a
+    bitmap.  Returns int [B, Hq, ceil(nQp / 2)], and the same count without the
+    skips (key tiles some query tile of the CTA visits)."""
+    from oracle import visited_tiles
+    B, Hq, nQ, _ = sb_words.shape
+    nK = -(-Lk // Bc)
+    skip = _unpack(sb_words, nK)
+    vis = np.zeros((nQ, nK), bool)
+    for qt in range(nQ):
+        vis[qt, :visited_tiles(causal, Lq, Lk, Br, Bc, qt)] = True
+    visit = np.broadcast_to(vis[None, None], skip.shape)
+    if selected is not None:
+        visit = visit & selected
+    per = 256 // Br
+    npairs = -(-(-(-Lq // 128)) // 2)
+
+    def per_cta(x):
+        pad = np.zeros((B, Hq, npairs * per, nK), bool)
+        pad[:, :, :nQ] = x
+        return pad.reshape(B, Hq, npairs, per, nK).any(axis=3).sum(axis=-1)
+
+    return per_cta(visit & ~skip), per_cta(visit)
+
+
 def gpu_run(q, k, v, *, causal, scale, mode, lam=0.0, n=0, m=0, sink=0, recent=0, Br=128, Bc=128,
             keep_bits=False):
+    """The kernel's outputs with its evidence: per-tile skip bits, keep bits
+    (optional), and V tile loads per CTA, which must equal the key tiles the
+    CTA's query tiles kept (a tile skipped by all of them loads no V)."""
     from softmax_ssa_fwd_b200 import ssa
     B, Lq, Hq, d = q.shape
     Lk = k.shape[1]
     nQ, nK = -(-Lq // Br), -(-Lk // Bc)
     sb = torch.zeros(B, Hq, nQ, -(-nK // 32), dtype=torch.int32, device=q.device)
     kb = torch.zeros(B, Hq, Lq, -(-Lk // 32), dtype=torch.int32, device=q.device) if keep_bits else None
+    npairs = -(-(-(-Lq // 128)) // 2)
+    vl = torch.full((B, Hq, npairs), -1, dtype=torch.int32, device=q.device)
     out, lse, cnt = ssa.attention(q, k, v, causal=causal, scale=scale, mode=mode, lam=lam, n=n, m=m,
-                                  sink=sink, recent=recent, Br=Br, Bc=Bc, skip_bits=sb, keep_bits=kb)
+                                  sink=sink, recent=recent, Br=Br, Bc=Bc, skip_bits=sb, keep_bits=kb,
+                                  v_tile_loads=vl)
     st = ssa.ssa_device_status()
     assert st == ssa.SSA_OK, ssa.status_string(st)
+    want, walked = expected_v_loads(sb.cpu().numpy().view(np.uint32), causal, Lq, Lk, Br, Bc)
+    got = vl.cpu().numpy()
+    assert np.array_equal(got, want), (
+        f"V tile loads differ from the kept tiles at {np.argwhere(got != want)[:8].tolist()}")
+    V_LOADS.append((os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], int(got.sum()),
+                    int(walked.sum())))
     return out, lse, cnt, sb, kb
 
 

@@ -30,7 +30,8 @@ def test_header_declares_the_entry_points():
     assert _declared_functions() == sorted(
         ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
          "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version",
-         "ssa_decode", "ssa_decode_workspace_bytes", "ssa_decode_default_splits", "ssa_fwd_blockmask"])
+         "ssa_decode", "ssa_decode_debug", "ssa_decode_workspace_bytes", "ssa_decode_default_splits",
+         "ssa_fwd_blockmask", "ssa_fwd_blockmask_debug"])
 
 
 def test_library_exports_every_declared_symbol(ssa):
@@ -65,7 +66,8 @@ def _call(ssa, **over):
     dict(B=0), dict(Hq=0), dict(Hkv=0), dict(Lq=0), dict(Lk=-3), dict(d=0),
     dict(Hq=6, Hkv=4), dict(scale=0.0), dict(scale=float("nan")), dict(scale=float("inf")),
     dict(lam=-1.0), dict(lam=float("nan")), dict(lam=float("inf")), dict(mode=4), dict(mode=-1),
-    dict(mode=2, sink=-1), dict(mode=3, recent=-5), dict(q=0x1008),
+    dict(mode=2, sink=-1), dict(mode=3, recent=-5), dict(q=0x1008), dict(cnt=0x6002),
+    dict(lse=0x5004),
 ])
 def test_invalid_arguments(ssa, over):
     assert _call(ssa, **over) == ssa.SSA_ERR_INVALID_ARG
@@ -181,3 +183,21 @@ def test_blockmask_argument_checks(ssa):
     assert ssa.lib.ssa_fwd_blockmask(*base, 0x7002, None) == ssa.SSA_ERR_INVALID_ARG    # misaligned
     long = base[:10] + (2049 * 128,) + base[11:]
     assert ssa.lib.ssa_fwd_blockmask(*long, 0x7000, None) == ssa.SSA_ERR_UNSUPPORTED   # > 2048 key tiles
+
+
+def test_debug_outputs_argument_checks(ssa):
+    base = (0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 1, 4, 2, 256, 256, 128, 1, 0.088, 1,
+            1e-3, 2, 4, 4, 128, 128, 128)
+    # misaligned 32-bit evidence outputs are refused before anything runs
+    assert ssa.lib.ssa_fwd_debug(*base, None, 0x7002, None, None) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.lib.ssa_fwd_debug(*base, None, None, 0x7001, None) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.lib.ssa_fwd_debug(*base, None, None, None, 0x7003) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.lib.ssa_fwd_blockmask_debug(*base, 0x7000, None, 0x8002, None) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.lib.ssa_fwd_blockmask_debug(*base, 0x7000, None, None, 0x8002) == ssa.SSA_ERR_INVALID_ARG
+    assert ssa.lib.ssa_fwd_blockmask_debug(*base, None, None, 0x8000, None) == ssa.SSA_ERR_INVALID_ARG
+    dec = (0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 2, 8, 2, 1, 4096, 128, 1, 0.088, 1e-4, 128,
+           4, 0x7000, ssa.ssa_decode_workspace_bytes(2, 8, 1, 128, 4), None)
+    assert ssa.lib.ssa_decode_debug(*dec, None) == ssa.SSA_ERR_INVALID_ARG          # no skip bits
+    assert ssa.lib.ssa_decode_debug(*dec, 0x9002) == ssa.SSA_ERR_INVALID_ARG        # misaligned
+    bad_cnt = dec[:5] + (0x6002,) + dec[6:]
+    assert ssa.lib.ssa_decode(*bad_cnt) == ssa.SSA_ERR_INVALID_ARG

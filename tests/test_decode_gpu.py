@@ -1,8 +1,9 @@
 """GPU parity of the split-KV decode path (ssa_decode through the C ABI)
 against the fp64 decode oracle (oracle/decode.py), on the same seeded bf16
 inputs: outputs max-abs <= 2e-2 and relative L2 <= 5e-3, lse max-abs <= 1e-3,
-per-head skip counts equal except tiles whose decision margin is within
-1e-3 * lambda (the oracle marks them)."""
+per-tile skip bits (ssa_decode_debug) identical -- a tile decided the other way
+inside the 1e-3 * lambda band (the oracle marks them) is taken the kernel's way
+in an oracle re-run, and there may be few -- and per-head skip counts equal."""
 import numpy as np
 import pytest
 import torch
@@ -30,16 +31,32 @@ def _gen(B, Hq, Hkv, Lq, Lk, d, seed, sink_coef):
 
 def _check(q, k, v, *, causal, scale, lam, Bc, splits, heads=None):
     from softmax_ssa_fwd_b200 import ssa
+    B, Lq, Hq, d = q.shape
+    nK = -(-k.shape[1] // Bc)
+    sb = torch.zeros(B, Hq, -(-nK // 32), dtype=torch.int32, device="cuda")
     out, lse, cnt = ssa.decode(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale, lam=lam,
-                               Bc=Bc, num_splits=splits)
+                               Bc=Bc, num_splits=splits, skip_bits=sb)
     assert ssa.ssa_device_status() == ssa.SSA_OK  # no bounded wait in the kernels gave up
-    ref = decode_oracle(q, k, v, causal=causal, scale=scale, lam=lam, Bc=Bc, num_splits=splits,
-                        heads=heads)
+    g_skip = np.unpackbits(sb.cpu().numpy().view(np.uint8), axis=-1, bitorder="little")[..., :nK].astype(bool)
+    pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    flip = np.zeros((B, Hq, nK), bool)
+    for _ in range(nK + 1):
+        ref = decode_oracle(q, k, v, causal=causal, scale=scale, lam=lam, Bc=Bc, num_splits=splits,
+                            heads=heads, flip=flip)
+        again = False
+        for b, h in pairs:
+            diff = g_skip[b, h] != ref.skip_bits[b, h]
+            if diff.any():
+                kt = int(np.argmax(diff))
+                assert ref.marginal[b, h, kt], f"skip decision differs outside the band at {(b, h, kt)}"
+                flip[b, h, kt] = True
+                again = True
+        if not again:
+            break
+    assert flip.sum() <= max(2, 5e-3 * len(pairs) * nK), flip.sum()
     o = out.float().cpu().numpy()
     ls = lse.cpu().numpy()
     c = cnt.cpu().numpy()
-    B, Lq, Hq, d = q.shape
-    pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hq)]
     num = den = 0.0
     worst = 0.0
     for b, h in pairs:
@@ -51,8 +68,7 @@ def _check(q, k, v, *, causal, scale, lam, Bc, splits, heads=None):
         assert np.array_equal(fin, np.isfinite(ls[b, h])), (b, h)
         if fin.any():
             assert np.abs(ls[b, h][fin] - ref.lse[b, h][fin]).max() <= LSE_MAX_ABS, (b, h)
-        margin = int(ref.marginal[b, h].sum())
-        assert abs(int(c[b, h]) - int(ref.skip_count[b, h])) <= margin, (b, h, c[b, h], ref.skip_count[b, h])
+        assert int(c[b, h]) == int(ref.skip_count[b, h]) == int(g_skip[b, h].sum()), (b, h)
     assert worst <= OUT_MAX_ABS, worst
     assert (num / max(den, 1e-30)) ** 0.5 <= OUT_REL_L2
     return ref, c

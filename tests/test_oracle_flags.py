@@ -330,3 +330,23 @@ def test_flip_is_accepted_only_inside_the_band():
     with pytest.raises(ValueError):
         run_items(q, k, v, causal=False, scale=1.0, mode=MODE_SKIP, lam=_lambda(case), Br=2, Bc=1,
                   flip_bits=flip)
+
+
+def test_decode_and_blockmask_flip_only_inside_the_band():
+    case = MARGIN_CASES[0]
+    q, k, v = _margin_inputs(case[0], case[1])
+    lam = _lambda(case)
+    flip = np.zeros((1, 1, 3), bool)
+    flip[0, 0, 1] = True
+    r = decode(q.view(1, 2, 1, D), k, v, causal=False, scale=1.0, lam=lam, Bc=1, num_splits=1, flip=flip)
+    assert r.skip_bits[0, 0].tolist() == [False, True, True]
+    words = np.full((1, 1, 1, 1), 0b111, np.uint32)
+    sb = np.zeros((1, 1, 1, 3), bool)
+    bm_oracle.run(q, k, v, words, causal=False, scale=1.0, lam=lam, Br=2, Bc=1, skip_bits=sb,
+                  flip=flip[:, :, None])
+    assert sb[0, 0, 0].tolist() == [False, True, True]
+    far = _lambda(MARGIN_CASES[2])
+    with pytest.raises(ValueError):
+        decode(q.view(1, 2, 1, D), k, v, causal=False, scale=1.0, lam=far, Bc=1, num_splits=1, flip=flip)
+    with pytest.raises(ValueError):
+        bm_oracle.run(q, k, v, words, causal=False, scale=1.0, lam=far, Br=2, Bc=1, flip=flip[:, :, None])

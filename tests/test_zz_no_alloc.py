@@ -9,12 +9,22 @@ kernel's status word, sits in a static device array inside the library.
 This file is named so pytest collects it last.  The test calls the entry
 point through the C ABI twice in a row (the shared scratch keeps the previous
 call's contents) and checks each result against ssa_fwd's on the same inputs,
-within the parity tolerance the other GPU tests use.
+within the parity tolerance the other GPU tests use, and against the fp64
+oracle.  A second test runs the entry point in a fresh process, before any
+allocating entry point, and checks that the device's free memory does not move
+across its calls; a third forces its bounded waits to give up and checks that
+the timeout is reported through ssa_device_status.
 """
 import math
+import os
+import subprocess
+import sys
 
+import numpy as np
 import pytest
 import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 pytestmark = pytest.mark.gpu
 
@@ -75,6 +85,80 @@ def test_noalloc_matches_ssa_fwd_twice_in_a_row():
     ref2 = _call(ssa.ssa_fwd, q2, k2, v2, 1e-3, mode=3, n=2, m=4, sink=4, recent=128)
     got2 = _call(ssa.ssa_fwd_noalloc, q2, k2, v2, 1e-3, mode=3, n=2, m=4, sink=4, recent=128)
     _close(got2, ref2)
+    # and the first problem's result against the fp64 oracle, every work item
+    from oracle import run_items
+    res = run_items(q.cpu(), k.cpu(), v.cpu(), causal=True, scale=1 / math.sqrt(q.shape[-1]), mode=1,
+                    lam=1e-2, Br=128, Bc=128)
+    o = second[0].float().cpu().numpy()
+    cnt = second[2].cpu().numpy()
+    L = q.shape[1]
+    for it, (b, h, t) in enumerate(res.items):
+        r0, r1 = t * 128, min(L, t * 128 + 128)
+        assert np.abs(o[b, r0:r1, h] - res.out[it, :r1 - r0]).max() <= OUT_MAX_ABS
+        assert int(cnt[b, h, t]) == int(res.skip_count[it])
+
+
+_FRESH = r"""
+import math, sys, torch
+sys.path.insert(0, ROOT)
+from softmax_ssa_fwd_b200 import ssa
+
+def inputs(seed, L, d):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(1, L, 8, d, generator=g); k = torch.randn(1, L, 2, d, generator=g)
+    v = torch.randn(1, L, 2, d, generator=g)
+    return [t.bfloat16().cuda() for t in (q, k, v)]
+
+def bufs(q):
+    B, L, Hq, d = q.shape
+    return (torch.empty_like(q), torch.empty(B, Hq, L, device="cuda"),
+            torch.empty(B, Hq, -(-L // 64), dtype=torch.int32, device="cuda"))
+
+def call(q, k, v, o, l, c, Bc):
+    B, L, Hq, d = q.shape
+    st = ssa.ssa_fwd_noalloc(q, k, v, o, l, c, B, Hq, 2, L, L, d, True, 1 / math.sqrt(d), 1, 1e-2,
+                             0, 0, 0, 0, 64, Bc, None)
+    assert st == ssa.SSA_OK, ssa.status_string(st)
+
+a = inputs(0, 700, 128); ba = bufs(a[0])
+b = inputs(1, 333, 64); bb = bufs(b[0])
+torch.cuda.synchronize()
+call(*a, *ba, 128)          # the first call on this device: looks up the scratch address
+torch.cuda.synchronize()
+free0 = torch.cuda.mem_get_info()[0]
+for _ in range(3):
+    call(*a, *ba, 128)
+call(*b, *bb, 64)           # another shape and another kernel instance
+assert ssa.ssa_device_status() == ssa.SSA_OK   # reads the status words, allocates nothing
+torch.cuda.synchronize()
+free1 = torch.cuda.mem_get_info()[0]
+print("free", free0, free1)
+assert free1 == free0, (free0, free1)
+"""
+
+
+def test_noalloc_first_in_a_fresh_process_leaves_free_memory_unchanged():
+    env = dict(os.environ, CUDA_MODULE_LOADING="EAGER")   # no kernel code loaded on first launch
+    r = subprocess.run([sys.executable, "-c", f"ROOT = {ROOT!r}\n" + _FRESH], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
+def test_noalloc_reports_a_timed_out_wait():
+    from softmax_ssa_fwd_b200 import ssa
+    q, k, v = _inputs(2)
+    ref = _call(ssa.ssa_fwd_noalloc, q, k, v, 1e-2)
+    assert ssa.ssa_device_status() == ssa.SSA_OK
+    try:
+        ssa.ssa_set_wait_timeout_ns(1)   # every pipeline wait gives up almost at once
+        _call(ssa.ssa_fwd_noalloc, q, k, v, 1e-2)
+        assert ssa.ssa_device_status() == ssa.SSA_ERR_TIMEOUT
+    finally:
+        ssa.ssa_set_wait_timeout_ns(0)
+    assert ssa.ssa_device_status() == ssa.SSA_OK   # read and cleared
+    again = _call(ssa.ssa_fwd_noalloc, q, k, v, 1e-2)
+    for x, y in zip(again, ref):
+        assert torch.equal(x, y)
 
 
 def test_noalloc_rejects_bad_arguments_synchronously():
