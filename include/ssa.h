@@ -160,6 +160,29 @@ int ssa_fwd_blockmask_debug(const void* q, const void* k, const void* v, void* o
                             int recent, int Br, int Bc, const uint32_t* block_mask, void* stream,
                             uint32_t* skip_bits, int32_t* v_tile_loads);
 
+/* Forward pass over caller-selected key blocks with proxy compensation of the
+ * omitted ones.  The PrimTS pull request page ("proxy compensation", "Bitmask
+ * format") keeps the selected blocks exact and stands in for every omitted
+ * KV block with two summaries the caller provides, the arithmetic mean of its
+ * keys and the sum of its values, correcting the softmax denominator by the
+ * number of tokens a summary represents (the true length of a final partial
+ * block included); a block computed exactly is not counted again.  The page
+ * gives no formula; this library reads it as: for query row i and an omitted
+ * block b of n_b keys, s_ib = scale * q_i . kmean_b adds n_b * exp(s_ib) to
+ * the denominator and exp(s_ib) * vsum_b to the numerator, as if each of its
+ * n_b keys had the mean key.  lse is the log of that denominator.
+ *   block_mask: as in ssa_fwd_blockmask (selects the exact blocks).
+ *   kmean, vsum: [B, nK, Hkv, d] bf16, 16-byte aligned, nK = ceil(Lk / Bc): per
+ *                key block (of Bc keys, the last one possibly shorter) the mean
+ *                of its keys and the sum of its values.
+ * Non-causal only, no skip-softmax and no N:M (SSA_ERR_UNSUPPORTED is not
+ * reachable: there is no causal or mode argument).  Other layouts, limits and
+ * status codes are those of ssa_fwd_blockmask; no skip counts are written. */
+int ssa_fwd_blockmask_proxy(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                            int Hq, int Hkv, int Lq, int Lk, int d, float scale, int Br, int Bc,
+                            const uint32_t* block_mask, const void* kmean, const void* vsum,
+                            void* stream);
+
 /* Total key tiles visited by all query tiles of one (batch, head) pair: a pure
  * function of the shape, used to turn skip counts into skip fractions and
  * executed FLOPs.  Returns -1 for invalid sizes. */

@@ -74,26 +74,32 @@ def run(q, k, v, mask_words, kmean, vsum, *, scale: float, Br: int, Bc: int, ite
     lse = np.full((B, Hq, Lq), -np.inf)
     if items is None:
         items = [(b, h, t) for b in range(B) for h in range(Hq) for t in range(nQ)]
+    qq = _as64(q)
     for b, hq, qt in items:
         hkv = hq // G
         kb, vb = _as64(k[b, :, hkv, :]), _as64(v[b, :, hkv, :])
+        # the terms of the query block: every key of a selected block, one
+        # (mean key, summed value, token count) term per omitted block
+        exact_keys, proxy_blocks, n_b = [], [], []
+        for blk in range(nK):
+            c0, c1 = blk * Bc, min(Lk, (blk + 1) * Bc)
+            if block_selected(mask_words, b, hkv, qt, blk):
+                exact_keys.extend(range(c0, c1))
+            else:
+                proxy_blocks.append(blk)
+                n_b.append(c1 - c0)
+        ke, ve = kb[exact_keys], vb[exact_keys]
+        kp, vp = km[b, proxy_blocks, hkv], vs[b, proxy_blocks, hkv]
+        n_b = np.array(n_b, dtype=np.float64)
         for i in range(qt * Br, min(Lq, qt * Br + Br)):
-            qi = _as64(q[b, i, hq, :])
-            # every term as (log weight, weighted value vector / weight)
-            logw, vals = [], []
-            for blk in range(nK):
-                c0, c1 = blk * Bc, min(Lk, (blk + 1) * Bc)
-                if block_selected(mask_words, b, hkv, qt, blk):
-                    for j in range(c0, c1):
-                        logw.append(scale * float(qi @ kb[j]))
-                        vals.append(vb[j])
-                else:
-                    n_b = c1 - c0
-                    logw.append(math.log(n_b) + scale * float(qi @ km[b, blk, hkv]))
-                    vals.append(vs[b, blk, hkv] / n_b)
-            mx = max(logw)
-            w = np.exp(np.array(logw) - mx)
+            qi = qq[b, i, hq, :]
+            # every term as a log weight and a value per unit of that weight:
+            # an exact key: s_ij and v_j; a proxy: log n_b + s_ib and vsum_b / n_b
+            logw = np.concatenate([scale * (ke @ qi), np.log(n_b) + scale * (kp @ qi)])
+            vals = np.concatenate([ve, vp / n_b[:, None]])
+            mx = logw.max()
+            w = np.exp(logw - mx)
             den = float(w.sum())
-            out[b, i, hq, :] = (w[:, None] * np.array(vals)).sum(axis=0) / den
+            out[b, i, hq, :] = (w[:, None] * vals).sum(axis=0) / den
             lse[b, hq, i] = mx + math.log(den)
     return out, lse

@@ -82,6 +82,9 @@ struct Params {
   float log2_lambda;  // -inf for lambda == 0
   unsigned long long wait_ns;  // limit of each pipeline wait
   const uint32_t* block_mask;  // optional [B, Hkv, nQ, nKw]: key blocks each query block visits
+  // proxy compensation of the omitted key blocks (bitmap variant only)
+  int nP;       // proxy steps: summary rows of all nK blocks in chunks of Bc
+  int n_last;   // keys in the final key block (its token mass)
 };
 
 struct __align__(8) Bars {
@@ -300,7 +303,8 @@ struct Work {
   int nvis;               // per CTA
 };
 
-// VAR: 0 plain, 1 with debug outputs (skip / keep bits), 2 key blocks selected by bitmap.
+// VAR: 0 plain, 1 with debug outputs (skip / keep bits), 2 key blocks selected by
+// bitmap, 3 key blocks selected by bitmap with proxy compensation of the others.
 template <int D, int BC, int NM_M, int VAR>
 __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b, int hq, int hkv,
                                              int t, int pt, int nvis_h0, int nvis_h1, int nsteps,
@@ -320,8 +324,9 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
   constexpr bool nm_on = NM_M != 0;
   const bool leader = p.half ? ((row & 63) == 0) : (row == 0);
   const int my_nvis = half ? nvis_h1 : nvis_h0;
-  constexpr bool DBG = VAR == 1, MASK = VAR == 2;
+  constexpr bool DBG = VAR == 1, MASK = VAR >= 2, PROXY = VAR == 3;
   const int nvis = nsteps;  // = max(nvis_h0, nvis_h1) unless key blocks are selected by bitmap
+  const int listed = MASK ? bars->listed : 0;  // exact steps, before the proxy steps
   const bool vote_on = skip_on || MASK;
 
   float m_true = -INFINITY;  // running max over kept tiles (raw q.k units)
@@ -337,14 +342,17 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     ok = __all_sync(0xffffffffu, ok);
     float m_tile = -INFINITY;
     // key tile of this step, and whether each logical query tile (half) of
-    // this tile visits it: visible, and selected when a bitmap is given
-    const int kt = MASK ? (int)bars->ktile[j] : j;
-    const int col0 = kt * BC;
+    // this tile visits it: visible, and selected when a bitmap is given.  A
+    // proxy step g covers the summaries of key blocks [g Bc, g Bc + Bc).
+    const bool is_proxy = PROXY && j >= listed;
+    const int kt = is_proxy ? j - listed : MASK ? (int)bars->ktile[j] : j;
+    const int col0 = kt * BC;  // first key (exact step) or first key block (proxy step)
     auto visits = [&](int h) -> bool {
       const int nv = h ? nvis_h1 : nvis_h0;
       if constexpr (!MASK) {
         return j < nv;
       } else {
+        if (is_proxy) return nv > 0;
         if (kt >= nv) return false;
         const int qt = p.half ? 2 * pt + h : pt;
         const uint32_t w = p.block_mask[((size_t)(b * p.Hkv + hkv) * p.nQ + qt) * p.nKw + (kt >> 5)];
@@ -360,12 +368,34 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     const bool nm_windows = nm_on && ((col0 < p.sink) ||
                                       (col0 <= pos_first + BM - 1 && col0 + BC - 1 > pos_first - p.recent));
     float x[BC];
+    // proxy step: the final key block's score (its token mass differs), -inf
+    // when it is not in this chunk or is computed exactly
+    float x_last = -INFINITY;
     // S from TMEM with the causal / length mask applied
     auto load_scores = [&]() {
 #pragma unroll
       for (int c = 0; c < BC / 32; ++c) tmem_ld32f(lane_base + s_col + 32 * c, &x[32 * c]);
+      const int c_last = p.nK - 1 - col0;
+      if (is_proxy && c_last < BC) x_last = tmem_ld1f(lane_base + s_col + c_last);
       tmem_wait_ld();
-      if (need_mask) {
+      if (is_proxy) {
+        // a block computed exactly by this query tile, or past the last
+        // block, contributes no proxy
+        const int qt = p.half ? 2 * pt + half : pt;
+        const uint32_t* mw = p.block_mask + ((size_t)(b * p.Hkv + hkv) * p.nQ + (qt < p.nQ ? qt : 0)) * p.nKw;
+#pragma unroll
+        for (int w = 0; w < BC / 32; ++w) {
+          const int wi = col0 / 32 + w;
+          uint32_t drop = (qt < p.nQ && wi < p.nKw) ? mw[wi] : 0xffffffffu;
+          const int left = p.nK - 32 * wi;  // blocks of this word that exist
+          if (left < 32) drop |= left <= 0 ? 0xffffffffu : (0xffffffffu << left);
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            if ((drop >> u) & 1u) x[32 * w + u] = -INFINITY;
+          if (c_last >= 32 * w && c_last < 32 * w + 32 && ((drop >> (c_last - 32 * w)) & 1u)) x_last = -INFINITY;
+        }
+        if (qt >= p.nQ) x_last = -INFINITY;
+      } else if (need_mask) {
         // last visible column of this row, relative to the tile
         int lim = p.Lk - 1 - col0;
         if (p.causal && pos - col0 < lim) lim = pos - col0;
@@ -519,7 +549,13 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       for (int bb = 1; bb < BC / 64; ++bb) p_block(bb);
       float ls0, ls1;
       f2_unpack(ls2, ls0, ls1);
-      l = l * alpha + (ls0 + ls1);
+      float ls = ls0 + ls1;
+      if (is_proxy) {
+        // every summary stands for Bc keys except the final block's n_last
+        ls = (float)BC * ls;
+        if (x_last != -INFINITY) ls -= (float)(BC - p.n_last) * mufu_exp2(fmaf(x_last, c, -mref_s));
+      }
+      l = l * alpha + ls;
       m_true = m_new;
       m_ref = m_ref_new;
     } else {
@@ -596,7 +632,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
   if (leader) {
     const int qt = p.half ? 2 * pt + half : pt;
     if (qt < p.nQ) {
-      p.skip_count[(size_t)(b * p.Hq + hq) * p.nQ + qt] = skipped;
+      if (p.skip_count != nullptr) p.skip_count[(size_t)(b * p.Hq + hq) * p.nQ + qt] = skipped;
       if (p.skip_bits != nullptr) {
         uint32_t* sb = p.skip_bits + ((size_t)(b * p.Hq + hq) * p.nQ + qt) * p.nKw;
         for (int w = (my_nvis + 31) / 32; w < p.nKw; ++w) sb[w] = 0u;
@@ -608,7 +644,8 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
 template <int D, int BC, int NM_M, int VAR>
 __global__ void __launch_bounds__(NTHREADS, 1)
     ssa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const Params p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_km,
+                   const __grid_constant__ CUtensorMap tm_vs, const Params p) {
   using L = Smem<D, BC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -622,7 +659,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const bool skip_on = (p.mode & SSA_MODE_SKIP) != 0;
   // the MMA warp and the V producer read the softmax's per-step keep bytes
   // whenever a tile may be left out: skip-softmax, or key blocks selected by bitmap
-  constexpr bool MASK = VAR == 2;
+  constexpr bool MASK = VAR >= 2, PROXY = VAR == 3;
   const bool vote_on = skip_on || MASK;
 
   // ---- work item: heaviest causal pairs first; query heads that share a KV
@@ -719,6 +756,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+    if (PROXY) {
+      tma_prefetch_desc(&tm_km);
+      tma_prefetch_desc(&tm_vs);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&bars->tmem_base), TMEM_COLS);
@@ -728,12 +769,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  const int listed = MASK ? bars->listed : 0;
   if (MASK) {
     wk.nvis_t[0] = bars->listed_t[0];
     wk.nvis_t[1] = bars->listed_t[1];
-    nvis = wk.nvis = bars->listed;
+    nvis = wk.nvis = listed;
   }
-  auto key_tile = [&](int j) { return MASK ? (int)bars->ktile[j] : j; };
+  if (PROXY) {
+    // no causal mask here: a query tile that exists visits every exact step,
+    // then every proxy step
+#pragma unroll
+    for (int t = 0; t < NQT; ++t) {
+      const bool exists = wk.nvis_h[t][0] > 0 || wk.nvis_h[t][1] > 0;
+      wk.nvis_t[t] = exists ? listed + p.nP : 0;
+    }
+    nvis = wk.nvis = listed + p.nP;
+  }
+  // key tile (or, for a proxy step, summary chunk) of step j, and its maps
+  auto key_tile = [&](int j) { return (PROXY && j >= listed) ? j - listed : MASK ? (int)bars->ktile[j] : j; };
+  auto k_map = [&](int j) { return (PROXY && j >= listed) ? &tm_km : &tm_k; };
+  auto v_map = [&](int j) { return (PROXY && j >= listed) ? &tm_vs : &tm_v; };
 
   if (warp < 4) {
     reg_dealloc<104>();
@@ -763,7 +818,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive_expect_tx(fb, L::K_BYTES);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(k_s + slot * L::K_BYTES + c * BC * 128, &tm_k, fb, c * 64, wk.hkv, key_tile(j) * BC, wk.b);
+          tma_load_4d(k_s + slot * L::K_BYTES + c * BC * 128, k_map(j), fb, c * 64, wk.hkv, key_tile(j) * BC, wk.b);
         issued = j + 1;
       }
       // drain: the newest load of each slot (older ones were consumed)
@@ -800,7 +855,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_arrive_expect_tx(fb, L::V_BYTES);
 #pragma unroll
             for (int c = 0; c < D / 64; ++c)
-              tma_load_4d(v_s + slot * L::V_BYTES + c * BC * 128, &tm_v, fb, c * 64, wk.hkv, key_tile(j) * BC, wk.b);
+              tma_load_4d(v_s + slot * L::V_BYTES + c * BC * 128, v_map(j), fb, c * 64, wk.hkv, key_tile(j) * BC, wk.b);
             last_load[slot] = j;
             loaded = true;
             ++n_loads;
@@ -946,7 +1001,7 @@ static unsigned long long g_wait_ns = WAIT_TIMEOUT_NS;
 static EncodeTiledFn g_encode = nullptr;
 constexpr int MAX_DEV = 64;
 static int* g_status[MAX_DEV] = {};
-static bool g_attr_set[MAX_DEV][36] = {};
+static bool g_attr_set[MAX_DEV][40] = {};
 
 static EncodeTiledFn encode_fn() {
   if (g_encode) return g_encode;
@@ -1000,9 +1055,12 @@ unsigned long long wait_timeout_ns() {
   return g_wait_ns;
 }
 
+struct Maps {
+  CUtensorMap q, k, v, km, vs;  // km / vs: proxy summaries (copies of k / v when unused)
+};
+
 template <int D, int BC, int NM_M, int VAR>
-static int launch_one(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                      const Params& p, int grid, cudaStream_t stream, int dev, int inst) {
+static int launch_one(const Maps& mp, const Params& p, int grid, cudaStream_t stream, int dev, int inst) {
   using L = Smem<D, BC>;
   if (!g_attr_set[dev][inst]) {
     if (cudaFuncSetAttribute(ssa_fwd_kernel<D, BC, NM_M, VAR>,
@@ -1010,30 +1068,29 @@ static int launch_one(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
       return SSA_ERR_CUDA;
     g_attr_set[dev][inst] = true;
   }
-  ssa_fwd_kernel<D, BC, NM_M, VAR><<<grid, NTHREADS, L::ALLOC, stream>>>(mq, mk, mv, p);
+  ssa_fwd_kernel<D, BC, NM_M, VAR><<<grid, NTHREADS, L::ALLOC, stream>>>(mp.q, mp.k, mp.v, mp.km, mp.vs, p);
   return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
 }
 
 // One instance per (N:M group width or none) x (plain, debug outputs, key
 // blocks by bitmap), so the plain skip-softmax kernel carries no N:M, debug or
-// bitmap code.
+// bitmap code; proxy compensation (no N:M) has one instance per shape.
 template <int D, int BC, int NM_M>
-static int launch_var(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                      const Params& p, int grid, cudaStream_t stream, int dev, int inst) {
-  if (p.block_mask != nullptr) return launch_one<D, BC, NM_M, 2>(mq, mk, mv, p, grid, stream, dev, inst + 2);
+static int launch_var(const Maps& mp, const Params& p, int grid, cudaStream_t stream, int dev, int inst) {
+  if (p.block_mask != nullptr) return launch_one<D, BC, NM_M, 2>(mp, p, grid, stream, dev, inst + 2);
   if (p.skip_bits != nullptr || p.keep_bits != nullptr || p.v_loads != nullptr)
-    return launch_one<D, BC, NM_M, 1>(mq, mk, mv, p, grid, stream, dev, inst + 1);
-  return launch_one<D, BC, NM_M, 0>(mq, mk, mv, p, grid, stream, dev, inst);
+    return launch_one<D, BC, NM_M, 1>(mp, p, grid, stream, dev, inst + 1);
+  return launch_one<D, BC, NM_M, 0>(mp, p, grid, stream, dev, inst);
 }
 
 template <int D, int BC>
-static int launch(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                  const Params& p, int grid, cudaStream_t stream, int dev, int base) {
+static int launch(const Maps& mp, const Params& p, int grid, cudaStream_t stream, int dev, int base) {
+  if (p.nP > 0) return launch_one<D, BC, 0, 3>(mp, p, grid, stream, dev, 36 + base);
   const int nm = (p.mode & SSA_MODE_NM) ? p.m : 0;
   const int inst = base * 9 + (nm == 0 ? 0 : nm == 4 ? 3 : 6);
-  if (nm == 0) return launch_var<D, BC, 0>(mq, mk, mv, p, grid, stream, dev, inst);
-  if (nm == 4) return launch_var<D, BC, 4>(mq, mk, mv, p, grid, stream, dev, inst);
-  return launch_var<D, BC, 8>(mq, mk, mv, p, grid, stream, dev, inst);
+  if (nm == 0) return launch_var<D, BC, 0>(mp, p, grid, stream, dev, inst);
+  if (nm == 4) return launch_var<D, BC, 4>(mp, p, grid, stream, dev, inst);
+  return launch_var<D, BC, 8>(mp, p, grid, stream, dev, inst);
 }
 
 static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -1044,9 +1101,13 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
                float scale, int mode, float lambda, int n, int m, int sink, int recent, int Br,
                int Bc, void* stream, uint32_t* skip_bits, uint32_t* keep_bits,
                int* status_override = nullptr, const uint32_t* block_mask = nullptr,
-               int32_t* v_loads = nullptr) {
+               int32_t* v_loads = nullptr, const void* kmean = nullptr, const void* vsum = nullptr) {
   // ---- argument checks (synchronous, nothing launched on failure)
-  if (!q || !k || !v || !out || !lse || !tile_skip_count) return SSA_ERR_INVALID_ARG;
+  const bool proxy = kmean != nullptr || vsum != nullptr;
+  if (!q || !k || !v || !out || !lse || (!tile_skip_count && !proxy)) return SSA_ERR_INVALID_ARG;
+  if (proxy && (!kmean || !vsum || !block_mask || !aligned16(kmean) || !aligned16(vsum)))
+    return SSA_ERR_INVALID_ARG;
+  if (proxy && (causal || mode != SSA_MODE_DENSE)) return SSA_ERR_UNSUPPORTED;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Lk <= 0 || d <= 0) return SSA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return SSA_ERR_INVALID_ARG;
   if (!std::isfinite(scale) || !(scale > 0.f)) return SSA_ERR_INVALID_ARG;
@@ -1076,15 +1137,24 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEV) return SSA_ERR_CUDA;
-  CUtensorMap mq, mk, mv;
+  Maps mp;
   Params p{};
+  const int nK = (Lk + Bc - 1) / Bc;
   {
     std::lock_guard<std::mutex> g(g_mu);
     p.status = status_override ? status_override : status_word(dev);
     if (!p.status) return SSA_ERR_CUDA;
-    if (!make_map(&mq, q, B, Lq, Hq, d, BM) || !make_map(&mk, k, B, Lk, Hkv, d, Bc) ||
-        !make_map(&mv, v, B, Lk, Hkv, d, Bc))
+    if (!make_map(&mp.q, q, B, Lq, Hq, d, BM) || !make_map(&mp.k, k, B, Lk, Hkv, d, Bc) ||
+        !make_map(&mp.v, v, B, Lk, Hkv, d, Bc))
       return SSA_ERR_CUDA;
+    if (proxy) {
+      // summaries [B, nK, Hkv, d]: one row per key block, loaded Bc rows at a time
+      if (!make_map(&mp.km, kmean, B, nK, Hkv, d, Bc) || !make_map(&mp.vs, vsum, B, nK, Hkv, d, Bc))
+        return SSA_ERR_CUDA;
+    } else {
+      mp.km = mp.k;
+      mp.vs = mp.v;
+    }
   }
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.lse = lse;
@@ -1110,16 +1180,18 @@ static int run(const void* q, const void* k, const void* v, void* out, float* ls
                                                            : -INFINITY;
   p.wait_ns = g_wait_ns;
   p.block_mask = block_mask;
+  p.nP = proxy ? (nK + Bc - 1) / Bc : 0;
+  p.n_last = Lk - (nK - 1) * Bc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // A caller-supplied status word (the allocation-free entry point's shared
   // scratch) keeps the previous call's contents: clear it on the stream first.
   if (status_override && cudaMemsetAsync(status_override, 0, sizeof(int), st) != cudaSuccess)
     return SSA_ERR_CUDA;
   std::lock_guard<std::mutex> g(g_mu);
-  if (d == 128 && Bc == 128) return launch<128, 128>(mq, mk, mv, p, (int)grid, st, dev, 0);
-  if (d == 128 && Bc == 64) return launch<128, 64>(mq, mk, mv, p, (int)grid, st, dev, 1);
-  if (d == 64 && Bc == 128) return launch<64, 128>(mq, mk, mv, p, (int)grid, st, dev, 2);
-  return launch<64, 64>(mq, mk, mv, p, (int)grid, st, dev, 3);
+  if (d == 128 && Bc == 128) return launch<128, 128>(mp, p, (int)grid, st, dev, 0);
+  if (d == 128 && Bc == 64) return launch<128, 64>(mp, p, (int)grid, st, dev, 1);
+  if (d == 64 && Bc == 128) return launch<64, 128>(mp, p, (int)grid, st, dev, 2);
+  return launch<64, 64>(mp, p, (int)grid, st, dev, 3);
 }
 
 
@@ -1214,6 +1286,15 @@ int ssa_fwd_blockmask_debug(const void* q, const void* k, const void* v, void* o
   return ssa::run(q, k, v, out, lse, tile_skip_count, B, Hq, Hkv, Lq, Lk, d, causal, scale, mode,
                   lambda, n, m, sink, recent, Br, Bc, stream, skip_bits, nullptr, nullptr, block_mask,
                   v_tile_loads);
+}
+
+int ssa_fwd_blockmask_proxy(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                            int Hq, int Hkv, int Lq, int Lk, int d, float scale, int Br, int Bc,
+                            const uint32_t* block_mask, const void* kmean, const void* vsum,
+                            void* stream) {
+  if (!block_mask || !kmean || !vsum) return SSA_ERR_INVALID_ARG;
+  return ssa::run(q, k, v, out, lse, nullptr, B, Hq, Hkv, Lq, Lk, d, 0, scale, SSA_MODE_DENSE, 0.f, 0, 0,
+                  0, 0, Br, Bc, stream, nullptr, nullptr, nullptr, block_mask, nullptr, kmean, vsum);
 }
 
 int64_t ssa_visited_tiles(int causal, int Lq, int Lk, int Br, int Bc) {

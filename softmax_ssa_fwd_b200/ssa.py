@@ -26,7 +26,7 @@ MODE_DENSE, MODE_SKIP, MODE_NM = 0, 1, 2
 EXPORTED = ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
             "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version",
             "ssa_decode", "ssa_decode_debug", "ssa_decode_workspace_bytes", "ssa_decode_default_splits",
-            "ssa_fwd_blockmask", "ssa_fwd_blockmask_debug"]
+            "ssa_fwd_blockmask", "ssa_fwd_blockmask_debug", "ssa_fwd_blockmask_proxy"]
 
 
 class SSAError(RuntimeError):
@@ -61,6 +61,8 @@ def _load():
     lib.ssa_fwd_blockmask.argtypes = fwd_args[:-1] + [P, P]
     lib.ssa_fwd_blockmask_debug.restype = I
     lib.ssa_fwd_blockmask_debug.argtypes = fwd_args[:-1] + [P, P, P, P]
+    lib.ssa_fwd_blockmask_proxy.restype = I
+    lib.ssa_fwd_blockmask_proxy.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, P, P, P]
     lib.ssa_decode.restype = I
     lib.ssa_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, F, I, I, P, ctypes.c_size_t, P]
     lib.ssa_decode_debug.restype = I
@@ -272,3 +274,27 @@ def attention_blockmask(q, k, v, block_mask, *, causal=True, scale=None, mode=MO
     if st != SSA_OK:
         raise SSAError(st, "ssa_fwd_blockmask")
     return out, lse, counts
+
+
+def ssa_fwd_blockmask_proxy(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, d, scale, Br, Bc, block_mask, kmean, vsum,
+                            stream=None) -> int:
+    """The proxy-compensated entry point (see include/ssa.h); returns its status code."""
+    return lib.ssa_fwd_blockmask_proxy(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lk, d,
+                                       float(scale), Br, Bc, _ptr(block_mask), _ptr(kmean), _ptr(vsum),
+                                       _stream(stream))
+
+
+def attention_blockmask_proxy(q, k, v, block_mask, kmean, vsum, *, scale=None, Br=128, Bc=128, stream=None):
+    """Selected key blocks exact, omitted ones through the caller's summaries
+    (kmean, vsum [B, nK, Hkv, d] bf16).  Returns (out, lse)."""
+    B, Lq, Hq, d = q.shape
+    _, Lk, Hkv, _ = k.shape
+    if scale is None:
+        scale = d ** -0.5
+    out = torch.empty_like(q)
+    lse = torch.empty(B, Hq, Lq, dtype=torch.float32, device=q.device)
+    st = ssa_fwd_blockmask_proxy(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, d, scale, Br, Bc, block_mask, kmean,
+                                 vsum, stream)
+    if st != SSA_OK:
+        raise SSAError(st, "ssa_fwd_blockmask_proxy")
+    return out, lse

@@ -31,7 +31,7 @@ def test_header_declares_the_entry_points():
         ["ssa_fwd", "ssa_fwd_debug", "ssa_fwd_noalloc", "ssa_visited_tiles",
          "ssa_set_wait_timeout_ns", "ssa_device_status", "ssa_status_string", "ssa_version",
          "ssa_decode", "ssa_decode_debug", "ssa_decode_workspace_bytes", "ssa_decode_default_splits",
-         "ssa_fwd_blockmask", "ssa_fwd_blockmask_debug"])
+         "ssa_fwd_blockmask", "ssa_fwd_blockmask_debug", "ssa_fwd_blockmask_proxy"])
 
 
 def test_library_exports_every_declared_symbol(ssa):
@@ -201,3 +201,15 @@ def test_debug_outputs_argument_checks(ssa):
     assert ssa.lib.ssa_decode_debug(*dec, 0x9002) == ssa.SSA_ERR_INVALID_ARG        # misaligned
     bad_cnt = dec[:5] + (0x6002,) + dec[6:]
     assert ssa.lib.ssa_decode(*bad_cnt) == ssa.SSA_ERR_INVALID_ARG
+
+
+def test_proxy_argument_checks(ssa):
+    base = (0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 1, 4, 2, 256, 256, 128, 0.088, 128, 128)
+    f = ssa.lib.ssa_fwd_blockmask_proxy
+    assert f(*base, None, 0x7000, 0x8000, None) == ssa.SSA_ERR_INVALID_ARG      # no mask
+    assert f(*base, 0x6000, None, 0x8000, None) == ssa.SSA_ERR_INVALID_ARG      # no kmean
+    assert f(*base, 0x6000, 0x7000, None, None) == ssa.SSA_ERR_INVALID_ARG      # no vsum
+    assert f(*base, 0x6000, 0x7008, 0x8000, None) == ssa.SSA_ERR_INVALID_ARG    # misaligned kmean
+    assert f(*base, 0x6000, 0x7000, 0x8004, None) == ssa.SSA_ERR_INVALID_ARG    # misaligned vsum
+    bad_d = base[:10] + (96,) + base[11:]
+    assert f(*bad_d, 0x6000, 0x7000, 0x8000, None) == ssa.SSA_ERR_UNSUPPORTED
