@@ -264,7 +264,37 @@ SWEEP = [
     ("stress wan local_alpha=2.5 lambda=1e-3", "wan", 1e-3, {"local_alpha": 2.5}),
     ("llama8k key blocks by bitmap density 0.25 lambda=1e-3", "llama8k", 1e-3, {"mask_density": 0.25}),
     ("decode qwen32k_decode lambda=1e-4", "qwen32k_decode", 1e-4, {}),
+    ("sol_proxy 84/512 exact blocks, proxy off", "sol_proxy", 0.0, {"exact_blocks": 84}),
+    ("sol_proxy 84/512 exact blocks, proxy on", "sol_proxy", 0.0, {"exact_blocks": 84, "proxy": True}),
 ]
+
+
+def exact_block_bits(w, per_row: int, seed: int) -> np.ndarray:
+    """Seeded selection of exactly per_row key blocks for every (batch, KV
+    head, query block): [B, Hkv, nQ, nK] bool."""
+    nQ, nK = -(-w.L // w.Br), -(-w.L // w.Bc)
+    rng = np.random.default_rng(seed)
+    bits = np.zeros((w.B, w.Hkv, nQ, nK), bool)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            for qt in range(nQ):
+                bits[b, h, qt, rng.choice(nK, size=per_row, replace=False)] = True
+    return bits
+
+
+def block_summaries_dev(k, v, Bc: int):
+    """The caller's proxy summaries on the device (input preparation, not
+    timed): per key block the mean of its keys and the sum of its values, bf16."""
+    B, L, H, d = k.shape
+    nK = -(-L // Bc)
+    pad = nK * Bc - L
+    kf = torch.nn.functional.pad(k.float(), (0, 0, 0, 0, 0, pad)).view(B, nK, Bc, H, d)
+    vf = torch.nn.functional.pad(v.float(), (0, 0, 0, 0, 0, pad)).view(B, nK, Bc, H, d)
+    cnt = torch.full((nK,), float(Bc), device=k.device)
+    cnt[-1] = Bc - pad
+    km = (kf.sum(dim=2) / cnt[None, :, None, None]).to(torch.bfloat16).contiguous()
+    vs = vf.sum(dim=2).to(torch.bfloat16).contiguous()
+    return km, vs
 
 
 def sweep_configs(dev, stream, target_ms: float = 400.0):
@@ -277,7 +307,9 @@ def sweep_configs(dev, stream, target_ms: float = 400.0):
     for label, name, lam, extra in SWEEP:
         w = WORKLOADS[name]
         dens = extra.get("mask_density", 0.0)
-        kw = {k_: v_ for k_, v_ in extra.items() if k_ != "mask_density"}
+        exact = extra.get("exact_blocks", 0)
+        proxy = extra.get("proxy", False)
+        kw = {k_: v_ for k_, v_ in extra.items() if k_ not in ("mask_density", "exact_blocks", "proxy")}
         if kw:
             w = w.with_(**kw)
         if w.Lq:  # decode
@@ -307,10 +339,18 @@ def sweep_configs(dev, stream, target_ms: float = 400.0):
             mask_bits = mask_dev = None
             if dens > 0:
                 mask_bits = block_mask_bits(w, dens, seed=w.seed)
+            if exact > 0:
+                mask_bits = exact_block_bits(w, exact, seed=w.seed)
+            if mask_bits is not None:
                 mask_dev = torch.from_numpy(pack_bits(mask_bits).view(np.int32)).to(dev)
+            summ = [block_summaries_dev(s_[1], s_[2], w.Bc) for s_ in sets] if proxy else None
 
             def launch(i):
                 q, k, v, o, l_, c = sets[i % nsets]
+                if proxy:
+                    km, vs = summ[i % nsets]
+                    return ssa.ssa_fwd_blockmask_proxy(q, k, v, o, l_, w.B, w.Hq, w.Hkv, w.L, w.L, w.d, w.scale,
+                                                       w.Br, w.Bc, mask_dev, km, vs, stream)
                 if mask_dev is not None:
                     return ssa.ssa_fwd_blockmask(q, k, v, o, l_, c, w.B, w.Hq, w.Hkv, w.L, w.L, w.d, w.causal,
                                                  w.scale, w.mode, lam, w.n, w.m, w.sink, w.recent, w.Br, w.Bc,
@@ -347,6 +387,20 @@ def sweep_configs(dev, stream, target_ms: float = 400.0):
                           "dense_equiv_tflops": dense_equiv_flops(w, Lq=w.Lq) / (ms * 1e-3) / 1e12,
                           "tiles_skipped_frac": skipped / visited,
                           "tokens_per_s": w.B * w.Lq / (ms * 1e-3)})
+        elif exact > 0:
+            # algorithmic work: the exact blocks (QK^T and P.V of Br x Bc x d each),
+            # plus, with proxies, one score and one P.V term of d per row and omitted block
+            nQ, nK = -(-w.L // w.Br), -(-w.L // w.Bc)
+            sel = float(mask_bits.sum()) * (w.Hq // w.Hkv)
+            fl = 4.0 * w.Br * w.Bc * w.d * sel
+            if proxy:
+                fl += 4.0 * w.d * w.B * w.Hq * w.L * (nK - exact)
+            entry.update({"algorithmic_tflops": fl / (ms * 1e-3) / 1e12,
+                          "algorithmic_frac_of_peak": fl / (ms * 1e-3) / 1e12 / bf16_peak,
+                          "tiles_skipped_frac": 0.0,
+                          "page_b200_ms": 1.2121 if proxy else 1.1261,
+                          "page_b200_ms_note": "the page's attention kernel p50 on its own B200 and data "
+                                               "(context, not the same inputs)"})
         else:
             visited = ssa.ssa_visited_tiles(w.causal, w.L, w.L, w.Br, w.Bc) * w.B * w.Hq
             if mask_bits is not None:

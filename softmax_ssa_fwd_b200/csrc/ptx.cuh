@@ -232,6 +232,19 @@ __device__ __forceinline__ void tmem_ld32f(uint32_t taddr, float* r) {
       : SSA_F8(0), SSA_F8(8), SSA_F8(16), SSA_F8(24)
       : "r"(taddr));
 }
+#define SSA_F64 SSA_F8(0), SSA_F8(8), SSA_F8(16), SSA_F8(24), SSA_F8(32), SSA_F8(40), SSA_F8(48), SSA_F8(56)
+// 64 consecutive 32-bit columns, fp32 (one instruction for a whole 64-column block).
+__device__ __forceinline__ void tmem_ld64f(uint32_t taddr, float* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : SSA_F64
+      : "r"(taddr));
+}
+#undef SSA_F64
 // 16 consecutive 32-bit columns, fp32.
 __device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float* r) {
   asm volatile(

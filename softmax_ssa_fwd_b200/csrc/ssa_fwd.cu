@@ -374,7 +374,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     // S from TMEM with the causal / length mask applied
     auto load_scores = [&]() {
 #pragma unroll
-      for (int c = 0; c < BC / 32; ++c) tmem_ld32f(lane_base + s_col + 32 * c, &x[32 * c]);
+      for (int c = 0; c < BC / 64; ++c) tmem_ld64f(lane_base + s_col + 64 * c, &x[64 * c]);
       const int c_last = p.nK - 1 - col0;
       if (is_proxy && c_last < BC) x_last = tmem_ld1f(lane_base + s_col + c_last);
       tmem_wait_ld();

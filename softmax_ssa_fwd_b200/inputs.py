@@ -18,6 +18,9 @@ Workloads (shapes from the pages' targets: Llama-3.1-8B / Qwen3-8B prefill in
                   3D RoPE over (t, h, w), seed 3, lambda = 1e-3
 * ``qwen32k``     B=2 Hq=32 Hkv=8 L=32768 d=128 causal, RoPE base 1e6, seed 4,
                   skip + N:M 2:4 (sink 4, recent 128), lambda = 1e-3
+* ``sol_proxy``   B=1 H=12 L=32760 d=128 non-causal, Br=Bc=64, seed 6: key
+                  blocks selected by bitmap (84 of 512 per query block, seeded
+                  at random), the others through proxy summaries
 * ``qwen32k_decode``  decode: B=8 sequences, one new query row each (the last
                   position) against L=32768 cached keys, Hq=32 Hkv=8 d=128,
                   RoPE base 1e6, seed 5, lambda = 1e-4 (the pages' decode
@@ -94,6 +97,11 @@ WORKLOADS = {
                     rope="3d", rope_base=1e4, sink_coef=0.0, grid=(21, 45, 80)),
     "qwen32k": Workload("qwen32k", 2, 32, 8, 32768, 128, True, 128, 128, MODE_SKIP | MODE_NM,
                         (1e-3,), n=2, m=4, sink=4, recent=128, seed=4, rope="1d", rope_base=1e6),
+    # block-sparse attention with proxy compensation, the shape of the PrimTS
+    # page's B200 measurement: [1, 32760, 12, 128], Q / KV blocks of 64, 84 of
+    # 512 key blocks exact per query block (no skip-softmax, non-causal)
+    "sol_proxy": Workload("sol_proxy", 1, 12, 12, 32760, 128, False, 64, 64, MODE_DENSE, (0.0,), seed=6,
+                          sink_coef=0.0),
     # decode phase: one new token per sequence against a 32k cache, 8 sequences,
     # the pages' decode threshold 1e-4; no N:M (prefill only)
     "qwen32k_decode": Workload("qwen32k_decode", 8, 32, 8, 32768, 128, True, 128, 128, MODE_SKIP,
