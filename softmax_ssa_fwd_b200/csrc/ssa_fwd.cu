@@ -59,6 +59,7 @@ constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;  // default limit of a pipel
 // loads, MMAs) finish before it frees its memory; never shortened.
 constexpr uint64_t DRAIN_TIMEOUT_NS = 2000000000ull;
 constexpr float RESCALE_LOG2 = 8.0f;  // lazy O rescale once the max grew by 2^8
+constexpr int VSLOTS = 4;             // vote slots per tile (see Bars::vote_bar)
 // Key tiles a CTA can list when the caller selects key blocks by bitmap.
 constexpr int MAX_LISTED_TILES = 2048;
 
@@ -92,10 +93,14 @@ struct __align__(8) Bars {
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
   uint64_t s_full[NQT], p_half[NQT], p_ready[NQT], o_done[NQT];
-  uint64_t vote_bar[NQT][2];  // per tile, per step parity: one arrival per softmax warp
+  // Votes of step j sit in slot j % VSLOTS (bytes and barrier phase j / VSLOTS).
+  // A tile's softmax runs at most two steps ahead of the V producer's read of
+  // its votes (the V producer may still read tile B's byte of step j after its
+  // V load released step j), so four slots never alias; two could.
+  uint64_t vote_bar[NQT][VSLOTS];  // per tile and slot: one arrival per softmax warp
   uint64_t mma_done;
   uint32_t tmem_base;
-  uint32_t vote[NQT][2];      // byte w: softmax warp w of the tile keeps the key tile
+  uint32_t vote[NQT][VSLOTS];      // byte w: softmax warp w of the tile keeps the key tile
   uint32_t abort_flag;
   int listed;                        // block-mask mode: key tiles in ktile[]
   int listed_t[NQT];                 // of which tile t visits the first listed_t[t]
@@ -461,12 +466,12 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     // The skip vote: each warp publishes one byte, "some row of mine keeps
     // the tile", and arrives on the tile's vote barrier for this step's
     // parity.  The MMA warp and the V producer read the same four bytes.
-    const uint32_t vbar = smem_u32(&bars->vote_bar[t][j & 1]);
+    const uint32_t vbar = smem_u32(&bars->vote_bar[t][j % VSLOTS]);
     bool wkeep = my_vis;
     if (vote_on) {
       wkeep = (skip_on ? !__all_sync(0xffffffffu, negligible) : true) && my_vis;
       if (lane == 0) {
-        st_shared_u8(smem_u32(&bars->vote[t][j & 1]) + quarter, wkeep ? 1u : 0u);
+        st_shared_u8(smem_u32(&bars->vote[t][j % VSLOTS]) + quarter, wkeep ? 1u : 0u);
         mbar_arrive(vbar);
       }
     }
@@ -479,12 +484,12 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
         // keeps it (the tile is skipped only if every row is negligible), so
         // it goes on at once; the other half's decision does not concern it.
         keep_h[0] = keep_h[1] = true;
-      } else if (!__all_sync(0xffffffffu, mbar_wait(vbar, (j >> 1) & 1, p.wait_ns))) {
+      } else if (!__all_sync(0xffffffffu, mbar_wait(vbar, (j / VSLOTS) & 1, p.wait_ns))) {
         // only a warp whose rows are all negligible waits for the others' votes
         if (!failed && lane == 0) record_failure(p, bars);
         failed = true;  // and keeps the tile
       } else {
-        const uint32_t w = ld_shared_u32(smem_u32(&bars->vote[t][j & 1]));
+        const uint32_t w = ld_shared_u32(smem_u32(&bars->vote[t][j % VSLOTS]));
         keep_h[0] = p.half ? (w & 0xffffu) != 0u : w != 0u;
         keep_h[1] = p.half ? (w >> 16) != 0u : w != 0u;
       }
@@ -743,8 +748,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int i = 0; i < NQT; ++i) {
       mbar_init(smem_u32(&bars->s_full[i]), 1);
-      mbar_init(smem_u32(&bars->vote_bar[i][0]), 4);
-      mbar_init(smem_u32(&bars->vote_bar[i][1]), 4);
+      for (int v = 0; v < VSLOTS; ++v) mbar_init(smem_u32(&bars->vote_bar[i][v]), 4);
       mbar_init(smem_u32(&bars->p_ready[i]), 4);  // one arrival per softmax warp
       mbar_init(smem_u32(&bars->p_half[i]), 4);
       mbar_init(smem_u32(&bars->o_done[i]), 1);
@@ -845,11 +849,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (j >= wk.nvis_t[t]) continue;
           bool keep = true;
           if (vote_on) {
-            if (!mbar_wait_fast(smem_u32(&bars->vote_bar[t][j & 1]), (j >> 1) & 1, p.wait_ns)) {
+            if (!mbar_wait_fast(smem_u32(&bars->vote_bar[t][j % VSLOTS]), (j / VSLOTS) & 1, p.wait_ns)) {
               fail = true;
               break;
             }
-            keep = ld_shared_u32(smem_u32(&bars->vote[t][j & 1])) != 0u;
+            keep = ld_shared_u32(smem_u32(&bars->vote[t][j % VSLOTS])) != 0u;
           }
           if (keep && !loaded) {
             mbar_arrive_expect_tx(fb, L::V_BYTES);
@@ -924,7 +928,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // P.V in two parts: the first 64 keys once their P is in TMEM, the
           // rest when the whole of P is
           if (!mbar_wait_fast(smem_u32(&bars->p_half[t]), j & 1, p.wait_ns)) { ok = false; break; }
-          const bool keep = !vote_on || ld_shared_u32(smem_u32(&bars->vote[t][j & 1])) != 0u;
+          const bool keep = !vote_on || ld_shared_u32(smem_u32(&bars->vote[t][j % VSLOTS])) != 0u;
           const uint32_t p_tmem = tmem + 256 * t;
           auto issue_pv = [&](int k0, int k1) {
             tc_fence_after();

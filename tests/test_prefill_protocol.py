@@ -8,164 +8,213 @@ for step j (or hands the slot on without a load); the MMA warp issues, per
 step j and tile, the first half of P.V once the softmax signals the first 64
 keys' P, the second half once all of P is written, then the tile's next
 QK^T; per tile four softmax warps read S, vote (one byte and one arrival per
-warp on the step parity's vote barrier), wait for the vote, rescale O when
-the running max grew (relying on S(j) completing after every earlier P.V of
-the tile), write P in two halves with a hand-off after each, and read O out
-at the end.  The tensor pipe runs in issue order; loads land in any order.
+warp in the step's vote slot, j mod 4; only a warp whose rows are all
+negligible waits for the others), rescale O when the running max grew
+(relying on S(j) completing after every earlier P.V of the tile), write P in
+two halves with a hand-off after each, and read O out at the end.  The tensor
+pipe runs in issue order; loads land in any order.
 
 Under random interleavings, speeds, visit counts (tile B visits one key tile
-more than A on causal diagonals, or none) and keep / rescale decisions, in
-skip mode and dense mode, every parity wait must see its own phase, nothing
-may deadlock, and the buffer hazards must hold: S read after its QK^T and
-overwritten only after every warp read it and its P.V ran; each half of a P.V
-reads a complete half of P and a landed V tile; K and V slots refilled only
-after their last reader; the vote bytes a reader sees are those of its step;
-O rescaled and read out only after every earlier P.V of its tile.
+more than A on causal diagonals, or none), per-warp votes and rescale
+decisions, in skip mode and dense mode, every parity wait must see its own
+phase, nothing may deadlock, and the buffer hazards must hold: S read after
+its QK^T and overwritten only after every warp read it and its P.V ran; each
+half of a P.V reads a complete half of P and a landed V tile; K and V slots
+refilled only after their last reader; the vote bytes a reader sees are those
+of its step; O rescaled and read out only after every earlier P.V of its
+tile.  With two vote slots instead of four some schedule breaks the last-but-
+one rule: after the V producer loads V_j on tile A's vote it still reads tile
+B's byte of step j, and a step both tiles skip lets the MMA warp issue tile
+B's QK^T two steps on, so tile B's softmax can overwrite that byte first.
+(The model walks a list of work items with its counters running across them;
+the kernel gives each CTA one.)
 """
 import random
 
 from protocol_model import Bar, ProtocolError, Sim
 
 KST, VST, NWARP, NQT = 2, 2, 4, 2
+VSLOTS = 4
 
 
 class Model(Sim):
-    def __init__(self, rng, nvis_t, keep, grow, vote_on):
+    def __init__(self, rng, items, vote_on, vslots=VSLOTS):
+        """items: list of (nvis_t [2], keep [2][n], grow [2][n], votes [2][n][NWARP])."""
         super().__init__(rng)
-        self.nvis_t = nvis_t          # key steps each query tile visits
-        self.nvis = max(nvis_t)
+        self.items = items
         self.vote_on = vote_on
-        # keep[t][j]: the tile's decision at step j (its first step is always kept)
-        self.keep = [[(not vote_on) or j == 0 or keep[t][j] for j in range(nvis_t[t])] for t in range(NQT)]
-        self.grow = grow
         B = Bar
-        self.q_full = B("q_full", 1)
+        self.q_full, self.q_empty = B("q_full", 1), B("q_empty", 1)
+        self.q_empty_wait = True
         self.k_full = [B(f"k_full{i}", 1) for i in range(KST)]
         self.k_empty = [B(f"k_empty{i}", 1) for i in range(KST)]
         self.v_full = [B(f"v_full{i}", 1) for i in range(VST)]
         self.v_empty = [B(f"v_empty{i}", 1) for i in range(VST)]
         self.s_full = [B(f"s_full{t}", 1) for t in range(NQT)]
-        self.vote_bar = [[B(f"vote_bar{t}{par}", NWARP) for par in range(2)] for t in range(NQT)]
+        self.vs = vslots
+        self.vote_bar = [[B(f"vote_bar{t}{v}", NWARP) for v in range(vslots)] for t in range(NQT)]
         self.p_half = [B(f"p_half{t}", NWARP) for t in range(NQT)]
         self.p_ready = [B(f"p_ready{t}", NWARP) for t in range(NQT)]
         self.o_done = [B(f"o_done{t}", 1) for t in range(NQT)]
-        n = self.nvis
-        self.q_landed = False
-        self.k_slot = [None] * KST
+        self.q_item = None                       # item whose Q tiles are in shared memory
+        self.k_slot = [None] * KST               # (item, step) a K slot holds
         self.v_slot = [None] * VST
-        self.qk_exec = [[False] * n for _ in range(NQT)]
-        self.s_read = [[0] * n for _ in range(NQT)]
-        self.p_blocks = [[[0, 0] for _ in range(n)] for _ in range(NQT)]
-        self.pv_exec = [[[False, False] for _ in range(n)] for _ in range(NQT)]
-        self.vote = [[None, None] for _ in range(NQT)]  # (step, bytes written) per parity
-        self.v_needed = [any(j < nvis_t[t] and self.keep[t][j] for t in range(NQT)) for j in range(n)]
+        self.qk = set()                          # (item, t, j) QK^T done
+        self.s_read = {}                         # (item, t, j) -> warps that read S
+        self.p_blocks = {}                       # (item, t, j) -> [warps done with half 0, half 1]
+        self.pv = {}                             # (item, t, j) -> [half 0 ran, half 1 ran]
+        self.vote = [[None] * vslots for _ in range(NQT)]   # per slot: (global step, bytes written)
+        self.o_read = set()                      # (item, t) epilogue read O
+        self.last_s = [None] * NQT               # (item, j) of tile t's newest S
+        self.live = [i for i, it in enumerate(items) if max(it[0]) > 0]
 
-    def users(self, j):
-        return [t for t in range(NQT) if j < self.nvis_t[t]]
+    def keep(self, n, t, j):
+        nvis_t, keep, _, _ = self.items[n]
+        return (not self.vote_on) or j == 0 or keep[t][j]
 
     # ------------------------------------------------------------ roles
     def qk_producer(self):
-        if self.nvis == 0:
-            return
-        yield ("tma", self.q_full, lambda: setattr(self, "q_landed", True))
-        for j in range(self.nvis):
-            if j >= KST:
-                yield ("wait", self.k_empty[j % KST], j // KST - 1)
-            yield ("do", lambda j=j: self.check(j < KST or all(self.qk_exec[t][j - KST] for t in self.users(j - KST)),
-                                                f"K slot of step {j} refilled before its last QK^T"))
-            yield ("tma", self.k_full[j % KST], lambda j=j: self.k_slot.__setitem__(j % KST, j))
+        gk, nq = 0, 0
+        for n in self.live:
+            nvis = max(self.items[n][0])
+            if nq > 0 and self.q_empty_wait:
+                yield ("wait", self.q_empty, nq - 1)
+            yield ("do", lambda n=n: self._check_q_free(n))
+            yield ("tma", self.q_full, lambda n=n: setattr(self, "q_item", n))
+            nq += 1
+            for j in range(nvis):
+                if gk >= KST:
+                    yield ("wait", self.k_empty[gk % KST], gk // KST - 1)
+                yield ("do", lambda gk=gk: self._check_k_free(gk))
+                yield ("tma", self.k_full[gk % KST], lambda n=n, j=j, gk=gk: self.k_slot.__setitem__(gk % KST, (n, j)))
+                gk += 1
 
     def v_producer(self):
-        for j in range(self.nvis):
-            slot = j % VST
-            if j >= VST:
-                yield ("wait", self.v_empty[slot], j // VST - 1)
-            loaded = False
-            for t in self.users(j):
-                keep = True
-                if self.vote_on:
-                    yield ("wait", self.vote_bar[t][j & 1], j >> 1)
-                    keep = self._read_vote(t, j, "V producer")
-                if keep and not loaded:
-                    yield ("do", lambda j=j: self._check_v_free(j))
-                    yield ("tma", self.v_full[slot], lambda j=j: self.v_slot.__setitem__(j % VST, j))
-                    loaded = True
-            if not loaded:
-                yield ("arrive", self.v_full[slot])
+        gv, gs = 0, [0, 0]
+        for n in self.live:
+            nvis_t = self.items[n][0]
+            for j in range(max(nvis_t)):
+                slot = gv % VST
+                if gv >= VST:
+                    yield ("wait", self.v_empty[slot], gv // VST - 1)
+                loaded = False
+                for t in range(NQT):
+                    if j >= nvis_t[t]:
+                        continue
+                    keep = True
+                    if self.vote_on:
+                        g = gs[t] + j
+                        yield ("wait", self.vote_bar[t][g % self.vs], g // self.vs)
+                        keep = self._read_vote(n, t, j, g, "V producer")
+                    if keep and not loaded:
+                        yield ("do", lambda gv=gv: self._check_v_free(gv))
+                        yield ("tma", self.v_full[slot], lambda n=n, j=j, s=slot: self.v_slot.__setitem__(s, (n, j)))
+                        loaded = True
+                if not loaded:
+                    yield ("arrive", self.v_full[slot])
+                gv += 1
+            for t in range(NQT):
+                gs[t] += nvis_t[t]
 
     def mma(self):
-        if self.nvis == 0:
-            return
-        yield ("wait", self.q_full, 0)
+        gk, gv, gs, nq = 0, 0, [0, 0], 0
         k_ready = [-1]
+        self.pv_slot_use = {}
+        for n in self.live:
+            nvis_t = self.items[n][0]
+            yield ("wait", self.q_full, nq)
+            nq += 1
+            qk_left = [sum(1 for t in range(NQT) if nvis_t[t] > 0)]
 
-        def issue_qk(t, j):
-            if k_ready[0] < j:
-                yield ("wait", self.k_full[j % KST], j // KST)
-                k_ready[0] = j
-            yield ("op", lambda t=t, j=j: self._exec_qk(t, j))
-            yield ("commit", self.s_full[t])
+            def issue_qk(t, j, gk=gk, n=n):
+                kg = gk + j
+                if k_ready[0] < kg:
+                    yield ("wait", self.k_full[kg % KST], kg // KST)
+                    k_ready[0] = kg
+                yield ("op", lambda: self._exec_qk(n, t, j, kg))
+                yield ("commit", self.s_full[t])
 
-        def k_last_user(j):
-            return 1 if j < self.nvis_t[1] else 0
+            def after_qk(t, j, gk=gk, nvis_t=nvis_t):
+                if (1 if j < nvis_t[1] else 0) == t:
+                    yield ("commit", self.k_empty[(gk + j) % KST])
+                if j == nvis_t[t] - 1:
+                    qk_left[0] -= 1
+                    if qk_left[0] == 0:
+                        yield ("commit", self.q_empty)
 
-        for t in range(NQT):
-            if self.nvis_t[t] > 0:
-                yield from issue_qk(t, 0)
-                if k_last_user(0) == t:
-                    yield ("commit", self.k_empty[0])
-        for j in range(self.nvis):
-            slot = j % VST
-            v_seen = any_pv = False
             for t in range(NQT):
-                if j >= self.nvis_t[t]:
-                    continue
-                yield ("wait", self.p_half[t], j)
-                keep = self._read_vote(t, j, "MMA") if self.vote_on else True
-                if keep:
-                    if not v_seen:
-                        yield ("wait", self.v_full[slot], j // VST)
-                        v_seen = True
-                    yield ("op", lambda t=t, j=j: self._exec_pv(t, j, 0))
-                yield ("wait", self.p_ready[t], j)
-                if keep:
-                    yield ("op", lambda t=t, j=j: self._exec_pv(t, j, 1))
-                    any_pv = True
-                if j == self.nvis_t[t] - 1:
-                    yield ("commit", self.o_done[t])
-                if j + 1 < self.nvis_t[t]:
-                    yield from issue_qk(t, j + 1)
-                    if k_last_user(j + 1) == t:
-                        yield ("commit", self.k_empty[(j + 1) % KST])
-            if not v_seen:
-                yield ("wait", self.v_full[slot], j // VST)
-            if any_pv:
-                yield ("commit", self.v_empty[slot])
-            else:
-                yield ("arrive", self.v_empty[slot])
+                if nvis_t[t] > 0:
+                    yield from issue_qk(t, 0)
+                    yield from after_qk(t, 0)
+            for j in range(max(nvis_t)):
+                slot = gv % VST
+                v_seen = any_pv = False
+                for t in range(NQT):
+                    if j >= nvis_t[t]:
+                        continue
+                    g = gs[t] + j
+                    yield ("wait", self.p_half[t], g)
+                    keep = self._read_vote(n, t, j, g, "MMA") if self.vote_on else True
+                    if keep:
+                        if not v_seen:
+                            yield ("wait", self.v_full[slot], gv // VST)
+                            v_seen = True
+                        yield ("op", lambda n=n, t=t, j=j, s=slot: self._exec_pv(n, t, j, 0, s))
+                    yield ("wait", self.p_ready[t], g)
+                    if keep:
+                        yield ("op", lambda n=n, t=t, j=j, s=slot: self._exec_pv(n, t, j, 1, s))
+                        any_pv = True
+                    if j == nvis_t[t] - 1:
+                        yield ("commit", self.o_done[t])
+                    if j + 1 < nvis_t[t]:
+                        yield from issue_qk(t, j + 1)
+                        yield from after_qk(t, j + 1)
+                if not v_seen:
+                    yield ("wait", self.v_full[slot], gv // VST)
+                if any_pv:
+                    yield ("commit", self.v_empty[slot])
+                else:
+                    yield ("arrive", self.v_empty[slot])
+                gv += 1
+            gk += max(nvis_t)
+            for t in range(NQT):
+                gs[t] += nvis_t[t]
 
     def softmax(self, t, w):
-        n_pv = 0
-        for j in range(self.nvis_t[t]):
-            yield ("wait", self.s_full[t], j)
-            yield ("do", lambda j=j: self._read_s(t, j))
-            keep = self.keep[t][j]
-            if self.vote_on:
-                yield ("do", lambda j=j: self._write_vote(t, j))
-                yield ("arrive", self.vote_bar[t][j & 1])
-                yield ("wait", self.vote_bar[t][j & 1], j >> 1)
-            if keep:
-                if self.grow[t][j] and n_pv > 0:
-                    yield ("do", lambda j=j: self._check_o(t, j, "rescaled"))
-                yield ("do", lambda j=j: self.p_blocks[t][j].__setitem__(0, self.p_blocks[t][j][0] + 1))
-            yield ("arrive", self.p_half[t])
-            if keep:
-                yield ("do", lambda j=j: self.p_blocks[t][j].__setitem__(1, self.p_blocks[t][j][1] + 1))
-                n_pv += 1
-            yield ("arrive", self.p_ready[t])
-        if self.nvis_t[t] > 0:
-            yield ("wait", self.o_done[t], 0)
-            yield ("do", lambda: self._check_o(t, self.nvis_t[t], "read out"))
+        gs, oi = 0, 0
+        for n in range(len(self.items)):
+            nvis_t, _, grow, votes = self.items[n]
+            n_pv = 0
+            for j in range(nvis_t[t]):
+                g = gs + j
+                yield ("wait", self.s_full[t], g)
+                yield ("do", lambda n=n, j=j: self._read_s(n, t, j))
+                keep = self.keep(n, t, j)
+                if self.vote_on:
+                    # a warp keeps when some row of it does; the tile keeps iff a warp does
+                    wkeep = votes[t][j][w] if keep else False
+                    if j == 0:
+                        wkeep = True
+                    yield ("do", lambda g=g: self._write_vote(t, g))
+                    yield ("arrive", self.vote_bar[t][g % self.vs])
+                    if not wkeep:
+                        yield ("wait", self.vote_bar[t][g % self.vs], g // self.vs)
+                        yield ("do", lambda n=n, j=j, g=g: self._read_vote(n, t, j, g, f"softmax{t}{w}"))
+                if keep:
+                    if grow[t][j] and n_pv > 0:
+                        yield ("do", lambda n=n, j=j: self._check_o(n, t, j, "rescaled"))
+                    yield ("do", lambda n=n, j=j: self._p_done(n, t, j, 0))
+                yield ("arrive", self.p_half[t])
+                if keep:
+                    yield ("do", lambda n=n, j=j: self._p_done(n, t, j, 1))
+                    n_pv += 1
+                yield ("arrive", self.p_ready[t])
+            if nvis_t[t] > 0:
+                yield ("wait", self.o_done[t], oi)
+                yield ("do", lambda n=n: self._check_o(n, t, self.items[n][0][t], "read out"))
+                yield ("do", lambda n=n: self.o_read.add((n, t, w)))
+                oi += 1
+            gs += nvis_t[t]
 
     def run(self):
         roles = [("qk_producer", self.qk_producer()), ("v_producer", self.v_producer()), ("mma", self.mma())]
@@ -173,70 +222,160 @@ class Model(Sim):
         Sim.run(self, roles)
 
     # ------------------------------------------------------------ state and checks
-    def _write_vote(self, t, j):
-        step, n = self.vote[t][j & 1] if self.vote[t][j & 1] and self.vote[t][j & 1][0] == j else (j, 0)
-        self.vote[t][j & 1] = (step, n + 1)
+    def _write_vote(self, t, g):
+        v = self.vote[t][g % self.vs]
+        step, cnt = v if v and v[0] == g else (g, 0)
+        self.vote[t][g % self.vs] = (step, cnt + 1)
 
-    def _read_vote(self, t, j, who):
-        v = self.vote[t][j & 1]
-        self.check(v is not None and v == (j, NWARP), f"{who} read tile {t}'s votes {v} at step {j}")
-        return self.keep[t][j]
+    def _read_vote(self, n, t, j, g, who):
+        v = self.vote[t][g % self.vs]
+        self.check(v is not None and v == (g, NWARP), f"{who} read tile {t}'s votes {v} at step {g}")
+        return self.keep(n, t, j)
 
-    def _check_v_free(self, j):
-        if j >= VST:
-            for t in self.users(j - VST):
-                if self.keep[t][j - VST]:
-                    self.check(all(self.pv_exec[t][j - VST]), f"V slot of step {j} refilled before the P.V of step {j - VST}")
+    def _check_q_free(self, n):
+        prev = [m for m in self.live if m < n]
+        if prev:
+            m = prev[-1]
+            nvis_t = self.items[m][0]
+            for t in range(NQT):
+                for j in range(nvis_t[t]):
+                    self.check((m, t, j) in self.qk, f"Q of item {n} loaded before QK^T({m},{t},{j}) ran")
 
-    def _exec_qk(self, t, j):
-        self.check(self.q_landed, "QK^T before the query tiles landed")
-        self.check(self.k_slot[j % KST] == j, f"QK^T({t},{j}) read a K slot holding step {self.k_slot[j % KST]}")
-        if j >= 1:
-            self.check(self.s_read[t][j - 1] == NWARP, f"S({t},{j}) overwrote S({t},{j - 1}) before every warp read it")
-            self.check(not self.keep[t][j - 1] or all(self.pv_exec[t][j - 1]),
-                       f"S({t},{j}) overwrote P({t},{j - 1}) before its P.V")
-        self.qk_exec[t][j] = True
+    def _check_k_free(self, gk):
+        if gk >= KST:
+            prev = self.k_slot[gk % KST]
+            self.check(prev is not None, "K slot refilled before its first load landed")
+            m, j = prev
+            for t in range(NQT):
+                if j < self.items[m][0][t]:
+                    self.check((m, t, j) in self.qk, f"K slot of ({m},{j}) refilled before QK^T({m},{t},{j})")
 
-    def _read_s(self, t, j):
-        self.check(self.qk_exec[t][j], f"softmax read S({t},{j}) before its QK^T ran")
-        self.s_read[t][j] += 1
+    def _check_v_free(self, gv):
+        if gv >= VST:
+            prev = self.v_slot[gv % VST]
+            if prev is not None:
+                m, j = prev
+                for t in range(NQT):
+                    if j < self.items[m][0][t] and self.keep(m, t, j):
+                        self.check(all(self.pv.get((m, t, j), [False, False])),
+                                   f"V slot of ({m},{j}) refilled before its P.V")
 
-    def _exec_pv(self, t, j, half):
-        self.check(self.p_blocks[t][j][half] == NWARP, f"P.V half {half} of ({t},{j}) read an incomplete P")
-        self.check(self.v_slot[j % VST] == j, f"P.V({t},{j}) read a V slot holding step {self.v_slot[j % VST]}")
-        self.pv_exec[t][j][half] = True
+    def _exec_qk(self, n, t, j, kg):
+        self.check(self.q_item == n, f"QK^T({n},{t},{j}) read Q tiles of item {self.q_item}")
+        self.check(self.k_slot[kg % KST] == (n, j), f"QK^T({n},{t},{j}) read a K slot holding {self.k_slot[kg % KST]}")
+        prev = self.last_s[t]
+        if prev is not None:
+            m, i = prev
+            self.check(self.s_read.get((m, t, i), 0) == NWARP, f"S({n},{t},{j}) overwrote S({m},{t},{i}) unread")
+            self.check(not self.keep(m, t, i) or all(self.pv.get((m, t, i), [False, False])),
+                       f"S({n},{t},{j}) overwrote P({m},{t},{i}) before its P.V")
+        self.last_s[t] = (n, j)
+        self.qk.add((n, t, j))
 
-    def _check_o(self, t, j, what):
+    def _read_s(self, n, t, j):
+        self.check((n, t, j) in self.qk, f"softmax read S({n},{t},{j}) before its QK^T ran")
+        self.s_read[(n, t, j)] = self.s_read.get((n, t, j), 0) + 1
+
+    def _p_done(self, n, t, j, half):
+        b = self.p_blocks.setdefault((n, t, j), [0, 0])
+        b[half] += 1
+
+    def _exec_pv(self, n, t, j, half, slot):
+        self.check(self.p_blocks.get((n, t, j), [0, 0])[half] == NWARP, f"P.V half {half} of ({n},{t},{j}) read an incomplete P")
+        self.check(self.v_slot[slot] == (n, j), f"P.V({n},{t},{j}) read a V slot holding {self.v_slot[slot]}")
+        if not any(self.pv.get((n, t, i), [False, False])[0] for i in range(j)) and half == 0:
+            # the item's first P.V of this tile overwrites O: the previous item's O must be read out
+            prev = [m for m in self.live if m < n and self.items[m][0][t] > 0]
+            if prev:
+                self.check(all((prev[-1], t, w) in self.o_read for w in range(NWARP)),
+                           f"first P.V of ({n},{t}) overwrote O of item {prev[-1]} before its epilogue read it")
+        self.pv.setdefault((n, t, j), [False, False])[half] = True
+
+    def _check_o(self, n, t, j, what):
         for h in range(j):
-            if self.keep[t][h]:
-                self.check(all(self.pv_exec[t][h]), f"O of tile {t} {what} at step {j} before the P.V of step {h}")
+            if self.keep(n, t, h):
+                self.check(all(self.pv.get((n, t, h), [False, False])),
+                           f"O of tile {t} of item {n} {what} at step {j} before the P.V of step {h}")
 
 
-def _random_case(rng):
-    a = rng.randint(0, 6)
-    b = rng.choice([a, a + 1, a + 1, 0 if a > 0 else 1])
-    nvis_t = [a, b]
-    keep = [[rng.random() < 0.6 for _ in range(8)] for _ in range(NQT)]
-    grow = [[rng.random() < 0.3 for _ in range(8)] for _ in range(NQT)]
-    return nvis_t, keep, grow, rng.random() < 0.8
+def _random_items(rng, count):
+    items = []
+    for _ in range(count):
+        a = rng.randint(0, 5)
+        b = rng.choice([a, a + 1, a + 1, 0 if a > 0 else 1])
+        nvis_t = [a, b]
+        keep = [[rng.random() < 0.6 for _ in range(8)] for _ in range(NQT)]
+        grow = [[rng.random() < 0.3 for _ in range(8)] for _ in range(NQT)]
+        votes = [[[rng.random() < 0.5 for _ in range(NWARP)] for _ in range(8)] for _ in range(NQT)]
+        for t in range(NQT):
+            for j in range(8):
+                if not any(votes[t][j]):
+                    votes[t][j][rng.randrange(NWARP)] = True   # a kept tile has a keeping warp
+        items.append((nvis_t, keep, grow, votes))
+    return items
 
 
 def test_prefill_protocol_holds_under_random_schedules():
-    runs = 0
     for seed in range(500):
         rng = random.Random(1000 + seed)
-        nvis_t, keep, grow, vote_on = _random_case(rng)
-        m = Model(rng, nvis_t, keep, grow, vote_on)
+        items = _random_items(rng, 1)   # the kernel gives each CTA one item
+        m = Model(rng, items, rng.random() < 0.8)
         m.run()
+        for n in m.live:
+            for t in range(NQT):
+                assert all((n, t, j) in m.qk for j in range(items[n][0][t])), seed
+
+
+def test_protocol_counters_run_across_items():
+    """The same roles walking several items with their counters running on
+    (q_empty guarding the query tiles) stay consistent as well."""
+    for seed in range(200):
+        rng = random.Random(5000 + seed)
+        Model(rng, _random_items(rng, rng.choice([2, 3, 4])), rng.random() < 0.8).run()
+
+
+def test_checker_finds_two_vote_slots_too_few():
+    found = 0
+    for seed in range(600):
+        rng = random.Random(seed)
+        # long items with many steps skipped by both tiles
+        items = _random_items(rng, 1)
+        items[0][0][0], items[0][0][1] = 7, 8
         for t in range(NQT):
-            assert all(m.qk_exec[t][:nvis_t[t]]), seed
-        runs += 1
-    assert runs == 500
+            items[0][1][t] = [j % 3 == 0 for j in range(8)]
+        try:
+            Model(rng, items, True, vslots=2).run()
+        except ProtocolError:
+            found += 1
+    assert found > 0
+
+
+def test_checker_finds_a_missing_q_empty_wait():
+    """Loading the next item's Q without waiting for the previous item's last
+    QK^T must be caught."""
+    class NoQEmpty(Model):
+        def qk_producer(self):
+            for cmd in Model.qk_producer(self):
+                if cmd[0] == "wait" and cmd[1] is self.q_empty:
+                    continue
+                yield cmd
+
+    found = 0
+    for seed in range(300):
+        rng = random.Random(seed)
+        items = _random_items(rng, 3)
+        for it in items:
+            it[0][0], it[0][1] = 2, 3
+        try:
+            NoQEmpty(rng, items, False).run()
+        except ProtocolError:
+            found += 1
+    assert found > 0
 
 
 def test_checker_finds_a_missing_p_half_wait():
-    """The same protocol with the MMA warp issuing the first half of P.V
-    without waiting for the softmax's first-half hand-off must be caught."""
+    """The MMA warp issuing the first half of P.V without waiting for the
+    softmax's first-half hand-off must be caught."""
     class NoHalfWait(Model):
         def mma(self):
             for cmd in Model.mma(self):
@@ -253,8 +392,10 @@ def test_checker_finds_a_missing_p_half_wait():
     found = 0
     for seed in range(300):
         rng = random.Random(seed)
+        items = _random_items(rng, 1)
+        items[0][0][0], items[0][0][1] = 4, 5
         try:
-            NoHalfWait(rng, [4, 5], [[True] * 8] * 2, [[False] * 8] * 2, True).run()
+            NoHalfWait(rng, items, False).run()
         except ProtocolError:
             found += 1
     assert found > 0
