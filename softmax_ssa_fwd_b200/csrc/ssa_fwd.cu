@@ -93,18 +93,24 @@ struct __align__(8) Bars {
   uint64_t k_full[KST], k_empty[KST];
   uint64_t v_full[VST], v_empty[VST];
   uint64_t s_full[NQT], p_half[NQT], p_ready[NQT], o_done[NQT];
-  // Votes of step j sit in slot j % VSLOTS (bytes and barrier phase j / VSLOTS).
-  // A tile's softmax runs at most two steps ahead of the V producer's read of
-  // its votes (the V producer may still read tile B's byte of step j after its
-  // V load released step j), so four slots never alias; two could.
+  // A tile's votes of its i-th step (counting the steps it takes part in) sit
+  // in slot i % VSLOTS (bytes and barrier phase i / VSLOTS).  A tile's softmax
+  // runs at most two of its steps ahead of the V producer's read of its votes
+  // (the V producer may still read tile B's byte of a step after its V load
+  // released that step), so four slots never alias; two could.
   uint64_t vote_bar[NQT][VSLOTS];  // per tile and slot: one arrival per softmax warp
   uint64_t mma_done;
   uint32_t tmem_base;
   uint32_t vote[NQT][VSLOTS];      // byte w: softmax warp w of the tile keeps the key tile
   uint32_t abort_flag;
   int listed;                        // block-mask mode: key tiles in ktile[]
-  int listed_t[NQT];                 // of which tile t visits the first listed_t[t]
+  int listed_t[NQT];                 // tile t takes part in no step from listed_t[t] on
   uint16_t ktile[MAX_LISTED_TILES];  // block-mask mode: the CTA's key tiles, ascending
+  // block-mask mode: bit 2t + h of part[j] is set when logical query tile
+  // (half) h of tile t selects and can see ktile[j]; tile t takes part in
+  // step j when either of its bits is.  Each tile's barrier phases and vote
+  // slots count only the steps it takes part in.
+  uint8_t part[MAX_LISTED_TILES];
 };
 
 template <int D, int BC>
@@ -353,14 +359,19 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
   uint32_t skip_word = 0;
   bool failed = false;
 
+  int step = 0;  // steps this tile took part in: its barrier phases and vote slots
   for (int j = 0; j < nvis; ++j) {
-    bool ok = !failed && mbar_wait(smem_u32(&bars->s_full[t]), j & 1, p.wait_ns);
-    ok = __all_sync(0xffffffffu, ok);
-    float m_tile = -INFINITY;
     // key tile of this step, and whether each logical query tile (half) of
     // this tile visits it: visible, and selected when a bitmap is given.  A
     // proxy step g covers the summaries of key blocks [g Bc, g Bc + Bc).
     const bool is_proxy = PROXY && j >= listed;
+    // with a bitmap, the tile takes part only in the listed steps it selects
+    const uint32_t pbits = (MASK && !is_proxy) ? ((uint32_t)bars->part[j] >> (2 * t)) & 3u : 3u;
+    if (pbits == 0u) continue;
+    const int i_step = MASK ? step++ : j;
+    bool ok = !failed && mbar_wait(smem_u32(&bars->s_full[t]), i_step & 1, p.wait_ns);
+    ok = __all_sync(0xffffffffu, ok);
+    float m_tile = -INFINITY;
     const int kt = is_proxy ? j - listed : MASK ? (int)bars->ktile[j] : j;
     const int col0 = kt * BC;  // first key (exact step) or first key block (proxy step)
     auto visits = [&](int h) -> bool {
@@ -369,10 +380,7 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
         return j < nv;
       } else {
         if (is_proxy) return nv > 0;
-        if (kt >= nv) return false;
-        const int qt = p.half ? 2 * pt + h : pt;
-        const uint32_t w = p.block_mask[((size_t)(b * p.Hkv + hkv) * p.nQ + qt) * p.nKw + (kt >> 5)];
-        return (w >> (kt & 31)) & 1u;
+        return (pbits >> (p.half ? h : 0)) & 1u;
       }
     };
     const bool vis0 = visits(0), vis1 = p.half ? visits(1) : vis0;
@@ -481,12 +489,12 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
     // The skip vote: each warp publishes one byte, "some row of mine keeps
     // the tile", and arrives on the tile's vote barrier for this step's
     // parity.  The MMA warp and the V producer read the same four bytes.
-    const uint32_t vbar = smem_u32(&bars->vote_bar[t][j % VSLOTS]);
+    const uint32_t vbar = smem_u32(&bars->vote_bar[t][i_step % VSLOTS]);
     bool wkeep = my_vis;
     if (vote_on) {
       wkeep = (skip_on ? !__all_sync(0xffffffffu, negligible) : true) && my_vis;
       if (lane == 0) {
-        st_shared_u8(smem_u32(&bars->vote[t][j % VSLOTS]) + quarter, wkeep ? 1u : 0u);
+        st_shared_u8(smem_u32(&bars->vote[t][i_step % VSLOTS]) + quarter, wkeep ? 1u : 0u);
         mbar_arrive(vbar);
       }
     }
@@ -499,12 +507,12 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
         // keeps it (the tile is skipped only if every row is negligible), so
         // it goes on at once; the other half's decision does not concern it.
         keep_h[0] = keep_h[1] = true;
-      } else if (!__all_sync(0xffffffffu, mbar_wait(vbar, (j / VSLOTS) & 1, p.wait_ns))) {
+      } else if (!__all_sync(0xffffffffu, mbar_wait(vbar, (i_step / VSLOTS) & 1, p.wait_ns))) {
         // only a warp whose rows are all negligible waits for the others' votes
         if (!failed && lane == 0) record_failure(p, bars);
         failed = true;  // and keeps the tile
       } else {
-        const uint32_t w = ld_shared_u32(smem_u32(&bars->vote[t][j % VSLOTS]));
+        const uint32_t w = ld_shared_u32(smem_u32(&bars->vote[t][i_step % VSLOTS]));
         keep_h[0] = p.half ? (w & 0xffffu) != 0u : w != 0u;
         keep_h[1] = p.half ? (w >> 16) != 0u : w != 0u;
       }
@@ -677,20 +685,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool skip_on = (p.mode & SSA_MODE_SKIP) != 0;
-  // the MMA warp and the V producer read the softmax's per-step keep bytes
-  // whenever a tile may be left out: skip-softmax, or key blocks selected by bitmap
+  // the MMA warp reads the softmax's per-step keep bytes whenever a tile may
+  // be left out (skip-softmax, or key blocks selected by bitmap, where one
+  // half of a 64-row pair may not select a key tile the other does); the V
+  // producer reads them only with skip-softmax
   constexpr bool MASK = VAR >= 2, PROXY = VAR == 3;
   const bool vote_on = skip_on || MASK;
 
-  // ---- work item: heaviest causal pairs first; query heads that share a KV
-  // head are adjacent in launch order.
+  // ---- work item.  Causal: heaviest pairs of query tiles first (the last
+  // pair visits the most key tiles), query heads that share a KV head
+  // adjacent.  Without a causal mask every pair costs the same: all pairs of
+  // one query head are adjacent, so the CTAs running at one time read the K
+  // and V of one or two heads, which stay in L2.
   Work wk;
   {
     const int per_pair = p.B * p.Hq;
     const int npairs = (p.nQp + 1) / 2;
-    int pair = blockIdx.x / per_pair;
-    if (p.causal) pair = npairs - 1 - pair;
-    const int bh = blockIdx.x % per_pair;
+    int pair, bh;
+    if (p.causal) {
+      pair = npairs - 1 - (int)(blockIdx.x / per_pair);
+      bh = blockIdx.x % per_pair;
+    } else {
+      pair = blockIdx.x % npairs;
+      bh = blockIdx.x / npairs;
+    }
     wk.b = bh / p.Hq;
     wk.hq = bh % p.Hq;
     wk.hkv = wk.hq / (p.Hq / p.Hkv);
@@ -714,7 +732,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   int nvis = wk.nvis;
 
   // ---- block-mask mode: the CTA walks the key tiles that any of its logical
-  // query tiles selects and can see, in ascending order (warp 3 lists them)
+  // query tiles selects and can see, in ascending order (warp 3 lists them
+  // with, per step, which logical query tiles take part)
   if (MASK && warp == 3) {
     int last[4], qts[4];
 #pragma unroll
@@ -724,29 +743,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       qts[x] = p.half ? 2 * wk.pt[t] + h : wk.pt[t];
     }
     const int maxlast = max(max(last[0], last[1]), max(last[2], last[3]));
-    const int last_t0 = max(last[0], last[1]), last_t1 = max(last[2], last[3]);
-    int count = 0, c0 = 0, c1 = 0;
+    int count = 0, end0 = 0, end1 = 0;
     for (int base = 0; base <= maxlast; base += 32) {
       const int kt = base + lane;
-      bool any = false;
+      uint32_t bits = 0;
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
         if (kt <= last[x]) {
           const uint32_t w = p.block_mask[((size_t)(wk.b * p.Hkv + wk.hkv) * p.nQ + qts[x]) * p.nKw + (kt >> 5)];
-          any |= ((w >> (kt & 31)) & 1u) != 0u;
+          bits |= ((w >> (kt & 31)) & 1u) << x;
         }
       }
-      const uint32_t bal = __ballot_sync(0xffffffffu, any);
+      const uint32_t bal = __ballot_sync(0xffffffffu, bits != 0u);
       const int pos = count + __popc(bal & ((1u << lane) - 1u));
-      if (any && pos < MAX_LISTED_TILES) bars->ktile[pos] = (uint16_t)kt;
+      if (bits != 0u && pos < MAX_LISTED_TILES) {
+        bars->ktile[pos] = (uint16_t)kt;
+        bars->part[pos] = (uint8_t)bits;
+      }
+      // one past each tile's last step so far: the listed lanes up to and
+      // including the highest lane in which the tile takes part
+      const uint32_t b0 = __ballot_sync(0xffffffffu, (bits & 3u) != 0u);
+      const uint32_t b1 = __ballot_sync(0xffffffffu, (bits & 12u) != 0u);
+      if (b0) end0 = count + __popc(bal & (0xffffffffu >> __clz(b0)));
+      if (b1) end1 = count + __popc(bal & (0xffffffffu >> __clz(b1)));
       count += __popc(bal);
-      c0 += __popc(__ballot_sync(0xffffffffu, any && kt <= last_t0));
-      c1 += __popc(__ballot_sync(0xffffffffu, any && kt <= last_t1));
     }
     if (lane == 0) {
       bars->listed = min(count, MAX_LISTED_TILES);
-      bars->listed_t[0] = min(c0, MAX_LISTED_TILES);
-      bars->listed_t[1] = min(c1, MAX_LISTED_TILES);
+      bars->listed_t[0] = min(end0, MAX_LISTED_TILES);
+      bars->listed_t[1] = min(end1, MAX_LISTED_TILES);
     }
   }
 
@@ -808,6 +833,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   auto key_tile = [&](int j) { return (PROXY && j >= listed) ? j - listed : MASK ? (int)bars->ktile[j] : j; };
   auto k_map = [&](int j) { return (PROXY && j >= listed) ? &tm_km : &tm_k; };
   auto v_map = [&](int j) { return (PROXY && j >= listed) ? &tm_vs : &tm_v; };
+  // tile t takes part in step j: the first nvis_t[t] steps, or with key blocks
+  // selected by bitmap the listed steps it selects (every proxy step when the
+  // tile exists)
+  auto part_of = [&](int t, int j) -> bool {
+    if constexpr (!MASK) {
+      return j < wk.nvis_t[t];
+    } else {
+      if (j >= wk.nvis_t[t]) return false;
+      if (PROXY && j >= listed) return true;
+      return ((bars->part[j] >> (2 * t)) & 3u) != 0u;
+    }
+  };
 
   if (warp < 4) {
     reg_dealloc<104>();
@@ -850,6 +887,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int last_load[VST];
       for (int i = 0; i < VST; ++i) last_load[i] = -1;
       int n_loads = 0;  // V tiles this CTA loaded (evidence output)
+      int step_t[NQT] = {0, 0};  // steps each tile took part in so far
       for (int j = 0; j < nvis; ++j) {
         if (aborted(bars)) break;
         const int slot = j % VST;
@@ -861,14 +899,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool loaded = false, fail = false;
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
-          if (j >= wk.nvis_t[t]) continue;
+          if (!part_of(t, j)) continue;
           bool keep = true;
-          if (vote_on) {
-            if (!mbar_wait_fast(smem_u32(&bars->vote_bar[t][j % VSLOTS]), (j / VSLOTS) & 1, p.wait_ns)) {
+          // Without skip-softmax a tile that takes part in a step keeps it (the
+          // rows of a query tile that selects the key tile vote to keep), so V
+          // is loaded at once; with it, only after the tile's votes are in.
+          if (skip_on) {
+            // the tile's own step count picks the vote slot and phase
+            const int i = MASK ? step_t[t]++ : j;
+            if (!mbar_wait_fast(smem_u32(&bars->vote_bar[t][i % VSLOTS]), (i / VSLOTS) & 1, p.wait_ns)) {
               fail = true;
               break;
             }
-            keep = ld_shared_u32(smem_u32(&bars->vote[t][j % VSLOTS])) != 0u;
+            keep = ld_shared_u32(smem_u32(&bars->vote[t][i % VSLOTS])) != 0u;
           }
           if (keep && !loaded) {
             mbar_arrive_expect_tx(fb, L::V_BYTES);
@@ -924,12 +967,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mma_commit(smem_u32(&bars->s_full[t]));
         return true;
       };
-      // last tile that reads K tile j: B when it visits j, else A
-      auto k_last_user = [&](int j) { return (j < wk.nvis_t[1]) ? 1 : 0; };
+      // last tile that reads K tile j: B when it takes part in step j, else A
+      auto k_last_user = [&](int j) { return part_of(1, j) ? 1 : 0; };
       int pv_count[NQT] = {0, 0};
+      int step_t[NQT] = {0, 0};  // steps each tile took part in so far
 #pragma unroll
       for (int t = 0; t < NQT; ++t)
-        if (ok && wk.nvis_t[t] > 0) {
+        if (ok && part_of(t, 0)) {
           ok = issue_qk(t, 0);
           if (ok && k_last_user(0) == t) mma_commit(smem_u32(&bars->k_empty[0]));
         }
@@ -939,11 +983,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool v_seen = false, any_pv = false;
 #pragma unroll
         for (int t = 0; t < NQT; ++t) {
-          if (j >= wk.nvis_t[t]) continue;
+          // a tile's next QK^T is issued while walking the step before it, so
+          // that it never waits on a K tile whose slot a later step frees
+          const bool next = j + 1 < nvis && part_of(t, j + 1);
+          if (!part_of(t, j)) {
+            if constexpr (MASK) {
+              if (next) {
+                if (!issue_qk(t, j + 1)) { ok = false; break; }
+                if (k_last_user(j + 1) == t) mma_commit(smem_u32(&bars->k_empty[(j + 1) % KST]));
+              }
+            }
+            continue;
+          }
+          // the tile's own step: barrier phases and vote slot (without a
+          // bitmap a tile takes part in a prefix of the steps)
+          const int i = MASK ? step_t[t]++ : j;
           // P.V in two parts: the first 64 keys once their P is in TMEM, the
           // rest when the whole of P is
-          if (!mbar_wait_fast(smem_u32(&bars->p_half[t]), j & 1, p.wait_ns)) { ok = false; break; }
-          const bool keep = !vote_on || ld_shared_u32(smem_u32(&bars->vote[t][j % VSLOTS])) != 0u;
+          if (!mbar_wait_fast(smem_u32(&bars->p_half[t]), i & 1, p.wait_ns)) { ok = false; break; }
+          const bool keep = !vote_on || ld_shared_u32(smem_u32(&bars->vote[t][i % VSLOTS])) != 0u;
           const uint32_t p_tmem = tmem + 256 * t;
           auto issue_pv = [&](int k0, int k1) {
             tc_fence_after();
@@ -960,14 +1018,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             issue_pv(0, 4);
           }
-          if (!mbar_wait_fast(smem_u32(&bars->p_ready[t]), j & 1, p.wait_ns)) { ok = false; break; }
+          if (!mbar_wait_fast(smem_u32(&bars->p_ready[t]), i & 1, p.wait_ns)) { ok = false; break; }
           if (keep) {
             issue_pv(4, BC / 16);
             ++pv_count[t];
             any_pv = true;
           }
           if (j == wk.nvis_t[t] - 1) mma_commit(smem_u32(&bars->o_done[t]));
-          if (j + 1 < wk.nvis_t[t]) {
+          if (next) {
             if (!issue_qk(t, j + 1)) { ok = false; break; }
             if (k_last_user(j + 1) == t) mma_commit(smem_u32(&bars->k_empty[(j + 1) % KST]));
           }
