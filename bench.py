@@ -578,6 +578,9 @@ def main():
     ap.add_argument("--mask-density", type=float, default=0.0,
                     help="select key blocks by a seeded random bitmap of this density "
                          "(ssa_fwd_blockmask); key tile 0 and the diagonal tile always selected")
+    ap.add_argument("--exact-blocks", type=int, default=0,
+                    help="select exactly this many key blocks per query block, seeded at random "
+                         "(ssa_fwd_blockmask; the selection the sol_proxy workload is measured with)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
@@ -615,7 +618,8 @@ def main():
     from softmax_ssa_fwd_b200 import ssa
 
     dev = torch.device("cuda", local_rank)
-    # two input sets, alternated between steps: 2 x 168 MB > 126 MB L2
+    # two input sets, alternated between steps (llama8k: 2 x 168 MB > 126 MB L2)
+    set_mb = 2 * (w.B * w.L * w.Hq * w.d + 2 * w.B * w.L * w.Hkv * w.d) / 1e6
     sets = []
     for s in range(2):
         q, k, v = make_inputs(w.with_(seed=w.seed + 1000 * s + 17 * rank), dev)
@@ -628,6 +632,9 @@ def main():
     mask_bits = mask_dev = None
     if args.mask_density > 0:
         mask_bits = block_mask_bits(w, args.mask_density, seed=w.seed + 31 * rank)
+    if args.exact_blocks > 0:
+        mask_bits = exact_block_bits(w, args.exact_blocks, seed=w.seed + 31 * rank)
+    if mask_bits is not None:
         mask_dev = torch.from_numpy(pack_bits(mask_bits).view(np.int32)).to(dev)
 
     def fwd(q, k, v, out, lse, cnt):
@@ -747,10 +754,12 @@ def main():
             "value": tflops_dense, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload_name(w, lam) + (f" key blocks by bitmap, density "
-                                                             f"{args.mask_density:g}" if mask_bits is not None else ""),
+            "config": {"workload": workload_name(w, lam) + (
+                           "" if mask_bits is None else
+                           f" key blocks by bitmap, {args.exact_blocks} of {nK} per query block" if args.exact_blocks
+                           else f" key blocks by bitmap, density {args.mask_density:g}"),
                        "parallelism": f"replicas x{world}",
-                       "l2": "inputs alternate between 2 sets of 168 MB each (> 126 MB L2)"},
+                       "l2": f"inputs alternate between 2 sets of {set_mb:.0f} MB each (Q, K, V; L2 126 MB)"},
             "executed_tflops": tflops_exec,
             "executed_frac_of_peak": tflops_exec / world / bf16_peak,
             "tiles_skipped_frac": skipped / visited,

@@ -13,7 +13,8 @@
 // One CTA owns two 128-row query tiles (A and B, adjacent in the sequence) of
 // one (batch, query head) and walks the key tiles they can see; K and V tiles
 // are loaded once for both.  Warp roles (384 threads):
-//   warp 0      Q and K producer: TMA into a KST-deep K ring
+//   warp 0      Q and K producer: TMA into a K ring (2 deep with 128 x 128
+//               tiles of K and V; 4 deep where shared memory allows)
 //   warp 1      TMEM owner and MMA issuer: S_t = Q_t K^T and O_t += P_t V on
 //               tcgen05, ping-ponging between the two tiles so the tensor pipe
 //               works on one tile while the other tile's softmax runs
@@ -50,8 +51,7 @@ namespace ssa {
 
 constexpr int BM = 128;       // rows per query tile = tcgen05 M
 constexpr int NQT = 2;        // query tiles per CTA
-constexpr int KST = 2;        // K ring depth
-constexpr int VST = 2;        // V ring depth
+constexpr int RING_MAX = 4;   // deepest K and V rings (see Smem)
 constexpr int NTHREADS = 384;
 constexpr int TMEM_COLS = 512;
 constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;  // default limit of a pipeline wait (2 s)
@@ -90,8 +90,8 @@ struct Params {
 
 struct __align__(8) Bars {
   uint64_t q_full;
-  uint64_t k_full[KST], k_empty[KST];
-  uint64_t v_full[VST], v_empty[VST];
+  uint64_t k_full[RING_MAX], k_empty[RING_MAX];
+  uint64_t v_full[RING_MAX], v_empty[RING_MAX];
   uint64_t s_full[NQT], p_half[NQT], p_ready[NQT], o_done[NQT];
   // A tile's votes of its i-th step (counting the steps it takes part in) sit
   // in slot i % VSLOTS (bytes and barrier phase i / VSLOTS).  A tile's softmax
@@ -118,12 +118,18 @@ struct Smem {
   static constexpr uint32_t QT_BYTES = BM * D * 2;  // one query tile
   static constexpr uint32_t K_BYTES = BC * D * 2;
   static constexpr uint32_t V_BYTES = BC * D * 2;
+  // K and V ring depths: four where both query tiles and four of each fit
+  // (64-key tiles, or d = 64), else two.  A step of a 64-key tile is short, so
+  // the loads need more steps of lead to hide their latency.
+  static constexpr int KST = (NQT * QT_BYTES + RING_MAX * (K_BYTES + V_BYTES) + 16384 <= 227u * 1024u) ? RING_MAX : 2;
+  static constexpr int VST = KST;
   static constexpr uint32_t Q_OFF = 0;
   static constexpr uint32_t K_OFF = Q_OFF + NQT * QT_BYTES;
   static constexpr uint32_t V_OFF = K_OFF + KST * K_BYTES;
   static constexpr uint32_t BAR_OFF = V_OFF + VST * V_BYTES;
   static constexpr uint32_t TOTAL = BAR_OFF + ((sizeof(Bars) + 127) / 128) * 128;
   static constexpr uint32_t ALLOC = TOTAL + 1024;  // slack for 1024-byte alignment
+  static_assert(ALLOC <= 227u * 1024u, "dynamic shared memory above the per-CTA limit");
 };
 
 // Key tiles visited by a logical query tile: all of them without a causal
@@ -675,6 +681,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_km,
                    const __grid_constant__ CUtensorMap tm_vs, const Params p) {
   using L = Smem<D, BC>;
+  constexpr int KST = L::KST, VST = L::VST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));

@@ -44,11 +44,12 @@ VSLOTS = 4
 
 
 class Model(Sim):
-    def __init__(self, rng, items, vote_on, vslots=VSLOTS, skip=True):
+    def __init__(self, rng, items, vote_on, vslots=VSLOTS, skip=True, kst=KST, vst=VST):
         """items: list of (part [2][n], keep [2][n], grow [2][n], votes [2][n][NWARP]);
         part[t][j]: tile t takes part in step j of the CTA's walk.  A list of two
         visit counts stands for the prefix pattern (tile t takes the first n_t)."""
         super().__init__(rng)
+        self.kst, self.vst = kst, vst   # ring depths (4 with 64-key tiles, where shared memory allows)
         self.items = [(_as_part(it[0]),) + tuple(it[1:]) for it in items]
         self.vote_on = vote_on
         # skip=False with votes on: key blocks by bitmap without skip-softmax.
@@ -59,10 +60,10 @@ class Model(Sim):
         B = Bar
         self.q_full, self.q_empty = B("q_full", 1), B("q_empty", 1)
         self.q_empty_wait = True
-        self.k_full = [B(f"k_full{i}", 1) for i in range(KST)]
-        self.k_empty = [B(f"k_empty{i}", 1) for i in range(KST)]
-        self.v_full = [B(f"v_full{i}", 1) for i in range(VST)]
-        self.v_empty = [B(f"v_empty{i}", 1) for i in range(VST)]
+        self.k_full = [B(f"k_full{i}", 1) for i in range(self.kst)]
+        self.k_empty = [B(f"k_empty{i}", 1) for i in range(self.kst)]
+        self.v_full = [B(f"v_full{i}", 1) for i in range(self.vst)]
+        self.v_empty = [B(f"v_empty{i}", 1) for i in range(self.vst)]
         self.s_full = [B(f"s_full{t}", 1) for t in range(NQT)]
         self.vs = vslots
         self.vote_bar = [[B(f"vote_bar{t}{v}", NWARP) for v in range(vslots)] for t in range(NQT)]
@@ -70,8 +71,8 @@ class Model(Sim):
         self.p_ready = [B(f"p_ready{t}", NWARP) for t in range(NQT)]
         self.o_done = [B(f"o_done{t}", 1) for t in range(NQT)]
         self.q_item = None                       # item whose Q tiles are in shared memory
-        self.k_slot = [None] * KST               # (item, step) a K slot holds
-        self.v_slot = [None] * VST
+        self.k_slot = [None] * self.kst               # (item, step) a K slot holds
+        self.v_slot = [None] * self.vst
         self.qk = set()                          # (item, t, j) QK^T done
         self.s_read = {}                         # (item, t, j) -> warps that read S
         self.p_blocks = {}                       # (item, t, j) -> [warps done with half 0, half 1]
@@ -105,19 +106,19 @@ class Model(Sim):
             yield ("tma", self.q_full, lambda n=n: setattr(self, "q_item", n))
             nq += 1
             for j in range(nsteps):
-                if gk >= KST:
-                    yield ("wait", self.k_empty[gk % KST], gk // KST - 1)
+                if gk >= self.kst:
+                    yield ("wait", self.k_empty[gk % self.kst], gk // self.kst - 1)
                 yield ("do", lambda gk=gk: self._check_k_free(gk))
-                yield ("tma", self.k_full[gk % KST], lambda n=n, j=j, gk=gk: self.k_slot.__setitem__(gk % KST, (n, j)))
+                yield ("tma", self.k_full[gk % self.kst], lambda n=n, j=j, gk=gk: self.k_slot.__setitem__(gk % self.kst, (n, j)))
                 gk += 1
 
     def v_producer(self):
         gv, gs = 0, [0, 0]   # gs[t]: tile t's steps so far (its vote slot and phase)
         for n in self.live:
             for j in range(_steps(self.items[n][0])):
-                slot = gv % VST
-                if gv >= VST:
-                    yield ("wait", self.v_empty[slot], gv // VST - 1)
+                slot = gv % self.vst
+                if gv >= self.vst:
+                    yield ("wait", self.v_empty[slot], gv // self.vst - 1)
                 loaded = False
                 for t in range(NQT):
                     if not self.part(n, t, j):
@@ -155,7 +156,7 @@ class Model(Sim):
             def issue_qk(t, j, gk=gk, n=n):
                 kg = gk + j
                 if k_ready[0] < kg:
-                    yield ("wait", self.k_full[kg % KST], kg // KST)
+                    yield ("wait", self.k_full[kg % self.kst], kg // self.kst)
                     k_ready[0] = kg
                 issued.add((t, j))
                 yield ("op", lambda: self._exec_qk(n, t, j, kg))
@@ -164,7 +165,7 @@ class Model(Sim):
             def after_qk(t, j, gk=gk, n=n):
                 # the last QK^T on K tile j: tile B's when B takes part in step j
                 if (1 if self.part(n, 1, j) else 0) == t:
-                    yield ("commit", self.k_empty[(gk + j) % KST])
+                    yield ("commit", self.k_empty[(gk + j) % self.kst])
                 if j == self.last(n, t):
                     qk_left[0] -= 1
                     if qk_left[0] == 0:
@@ -175,7 +176,7 @@ class Model(Sim):
                     yield from issue_qk(t, 0)
                     yield from after_qk(t, 0)
             for j in range(nsteps):
-                slot = gv % VST
+                slot = gv % self.vst
                 v_seen = any_pv = False
                 for t in range(NQT):
                     if self.part(n, t, j):
@@ -185,7 +186,7 @@ class Model(Sim):
                         keep = self._read_vote(n, t, j, g, "MMA") if self.vote_on else True
                         if keep:
                             if not v_seen:
-                                yield ("wait", self.v_full[slot], gv // VST)
+                                yield ("wait", self.v_full[slot], gv // self.vst)
                                 v_seen = True
                             yield ("op", lambda n=n, t=t, j=j, s=slot: self._exec_pv(n, t, j, 0, s))
                         yield ("wait", self.p_ready[t], g)
@@ -199,7 +200,7 @@ class Model(Sim):
                         yield from issue_qk(t, nxt)
                         yield from after_qk(t, nxt)
                 if not v_seen:
-                    yield ("wait", self.v_full[slot], gv // VST)
+                    yield ("wait", self.v_full[slot], gv // self.vst)
                 if any_pv:
                     yield ("commit", self.v_empty[slot])
                 else:
@@ -271,8 +272,8 @@ class Model(Sim):
                         self.check((m, t, j) in self.qk, f"Q of item {n} loaded before QK^T({m},{t},{j}) ran")
 
     def _check_k_free(self, gk):
-        if gk >= KST:
-            prev = self.k_slot[gk % KST]
+        if gk >= self.kst:
+            prev = self.k_slot[gk % self.kst]
             self.check(prev is not None, "K slot refilled before its first load landed")
             m, j = prev
             for t in range(NQT):
@@ -280,8 +281,8 @@ class Model(Sim):
                     self.check((m, t, j) in self.qk, f"K slot of ({m},{j}) refilled before QK^T({m},{t},{j})")
 
     def _check_v_free(self, gv):
-        if gv >= VST:
-            prev = self.v_slot[gv % VST]
+        if gv >= self.vst:
+            prev = self.v_slot[gv % self.vst]
             if prev is not None:
                 m, j = prev
                 for t in range(NQT):
@@ -291,7 +292,7 @@ class Model(Sim):
 
     def _exec_qk(self, n, t, j, kg):
         self.check(self.q_item == n, f"QK^T({n},{t},{j}) read Q tiles of item {self.q_item}")
-        self.check(self.k_slot[kg % KST] == (n, j), f"QK^T({n},{t},{j}) read a K slot holding {self.k_slot[kg % KST]}")
+        self.check(self.k_slot[kg % self.kst] == (n, j), f"QK^T({n},{t},{j}) read a K slot holding {self.k_slot[kg % self.kst]}")
         prev = self.last_s[t]
         if prev is not None:
             m, i = prev
@@ -466,6 +467,15 @@ def test_checker_finds_votes_counted_by_walk_step():
         except ProtocolError:
             found += 1
     assert found > 0
+
+
+def test_protocol_holds_with_four_deep_rings():
+    """The 4-deep K and V rings of the shapes whose tiles leave room for them."""
+    for seed in range(300):
+        rng = random.Random(7000 + seed)
+        sel = rng.random() < 0.5
+        Model(rng, _random_items(rng, 1, selected=sel), rng.random() < 0.8, skip=rng.random() < 0.7,
+              kst=4, vst=4).run()
 
 
 def test_protocol_counters_run_across_items():
