@@ -49,6 +49,10 @@ CASES = [
     (2, 8, 2, 512, 128, False, 128, 64, MODE_SKIP, 1e-3, 0.6, 3.0),
     (1, 4, 4, 600, 128, True, 128, 128, MODE_DENSE, 0.0, 0.5, 3.0),
     (1, 4, 2, 640, 128, True, 64, 128, MODE_SKIP, 0.0, 0.4, 6.0),
+    # 64-key blocks without skip-softmax: causal with a ragged last block, and
+    # d = 64 with a one-key last block
+    (1, 4, 2, 700, 128, True, 64, 64, MODE_DENSE, 0.0, 0.3, 3.0),
+    (2, 4, 4, 513, 64, False, 128, 64, MODE_DENSE, 0.0, 0.5, 3.0),
 ]
 
 
