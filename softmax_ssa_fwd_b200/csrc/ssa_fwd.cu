@@ -321,6 +321,35 @@ __device__ __forceinline__ void nm_by_rank(float (&x)[64], int N, int col0, int 
   }
 }
 
+// The exact-tie path of the N:M selection, out of line so that its registers
+// do not burden the softmax loop: one row of S (columns [0, BC) at s_addr)
+// from TMEM, the causal / length mask (columns past lim become -inf), the
+// rank-based selection, and the selected scores written back over S, from
+// where the caller reloads them.  Warp-collective (the caller's branch is
+// warp-uniform).
+template <int M, int BC>
+__device__ __noinline__ void nm_redo_in_tmem(uint32_t s_addr, int N, int col0, int lim, int pos, int sink,
+                                             int recent, bool windows) {
+#pragma unroll 1
+  for (int bb = 0; bb < BC / 64; ++bb) {
+    float x[64];
+    tmem_ld64f(s_addr + 64 * bb, x);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+      if (64 * bb + i > lim) x[i] = -INFINITY;
+    nm_by_rank<M>(x, N, col0 + 64 * bb, pos, sink, recent, windows);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t u[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(x[32 * h + i]);
+      tmem_st32(s_addr + 64 * bb + 32 * h, u);
+    }
+  }
+  tmem_wait_st();
+}
+
 struct Work {
   int b, hq, hkv;
   int pt[NQT];            // 128-row tile index of tile t
@@ -451,12 +480,29 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
         if (__any_sync(0xffffffffu, tie)) {
           // an exact tie at a group boundary in some row of this warp: the
           // whole warp starts again from the scores (still in TMEM; the
-          // tcgen05 load is warp-collective) and ranks explicitly
-          load_scores();
+          // tcgen05 accesses are warp-collective) and ranks explicitly.  With
+          // 128-key tiles that runs out of line, leaving the selected scores
+          // in place of S to be reloaded (inline, its registers made the
+          // loop spill: measured +3 % on 2:4, +7 % on 4:8); 64-key tiles, and
+          // the 1:4 instance (out of line it spills instead), redo it in
+          // registers.
+          if constexpr (BC == 128 && NM_M != 41) {
+            int lim = BC - 1;
+            if (need_mask) {
+              lim = p.Lk - 1 - col0;
+              if (p.causal && pos - col0 < lim) lim = pos - col0;
+            }
+            nm_redo_in_tmem<MM, BC>(lane_base + s_col, p.n, col0, lim, pos, p.sink, p.recent, nm_windows);
 #pragma unroll
-          for (int bb = 0; bb < BC / 64; ++bb)
-            nm_by_rank<MM>(*reinterpret_cast<float(*)[64]>(&x[64 * bb]), p.n, col0 + 64 * bb, pos,
-                           p.sink, p.recent, nm_windows);
+            for (int c = 0; c < BC / 64; ++c) tmem_ld64f(lane_base + s_col + 64 * c, &x[64 * c]);
+            tmem_wait_ld();
+          } else {
+            load_scores();
+#pragma unroll
+            for (int bb = 0; bb < BC / 64; ++bb)
+              nm_by_rank<MM>(*reinterpret_cast<float(*)[64]>(&x[64 * bb]), p.n, col0 + 64 * bb, pos,
+                             p.sink, p.recent, nm_windows);
+          }
         }
       }
       // four independent chains keep the dependent depth at BC / 8
