@@ -265,6 +265,32 @@ __device__ __forceinline__ bool nm8_fast(float (&x)[64], int N, int col0, int po
   return tie;
 }
 
+// 8-wide groups with N = 4: the 4th and 5th largest of a group from its two
+// sorted halves a, c (5 comparators each): the k-th largest of the union is
+// the largest, over i + j = k, of min(i-th largest of a, j-th largest of c)
+// (the 0-th being +inf).  32 min/max against 38 for a full sort plus the
+// run-time choice of N.
+template <bool WIN>
+__device__ __forceinline__ bool nm8_n4(float (&x)[64], int col0, int pos, int sink, int recent) {
+  bool tie = false;
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    float a[4], c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[i] = x[8 * g + i];
+      c[i] = x[8 * g + 4 + i];
+    }
+    sort_desc<4>(a);
+    sort_desc<4>(c);
+    const float t = fmaxf(fmax3(c[3], fminf(a[0], c[2]), fminf(a[1], c[1])), fmaxf(fminf(a[2], c[0]), a[3]));
+    const float nx = fmaxf(fmax3(fminf(a[0], c[3]), fminf(a[1], c[2]), fminf(a[2], c[1])), fminf(a[3], c[0]));
+    tie |= (t == nx) & (t != -INFINITY);
+    nm_keep_group<WIN>(&x[8 * g], 8, t, col0 + 8 * g, pos, sink, recent);
+  }
+  return tie;
+}
+
 template <int M, bool WIN>
 __device__ __forceinline__ bool nm_fast_w(float (&x)[64], int N, int col0, int pos, int sink, int recent) {
   if constexpr (M == 4) {
@@ -358,8 +384,8 @@ struct Work {
   int nvis;               // per CTA
 };
 
-// NM_M: 0 no N:M; 8 eight-wide groups (N at run time); 41, 42, 43 four-wide
-// groups with N = 1, 2, 3.
+// NM_M: 0 no N:M; 8 eight-wide groups (N at run time); 84 eight-wide groups
+// with N = 4; 41, 42, 43 four-wide groups with N = 1, 2, 3.
 // VAR: 0 plain, 1 with debug outputs (skip / keep bits), 2 key blocks selected by
 // bitmap, 3 key blocks selected by bitmap with proxy compensation of the others.
 template <int D, int BC, int NM_M, int VAR>
@@ -467,12 +493,15 @@ __device__ __forceinline__ void softmax_tile(const Params& p, Bars* bars, int b,
       tc_fence_after();
       load_scores();
       if constexpr (nm_on) {
-        constexpr int MM = NM_M >= 40 ? 4 : (NM_M ? NM_M : 4);  // group width
+        constexpr int MM = (NM_M == 8 || NM_M == 84) ? 8 : 4;  // group width
         bool tie = false;
 #pragma unroll
         for (int bb = 0; bb < BC / 64; ++bb) {
           auto& xb = *reinterpret_cast<float(*)[64]>(&x[64 * bb]);
-          if constexpr (NM_M >= 40)
+          if constexpr (NM_M == 84)
+            tie |= nm_windows ? nm8_n4<true>(xb, col0 + 64 * bb, pos, p.sink, p.recent)
+                              : nm8_n4<false>(xb, col0 + 64 * bb, pos, p.sink, p.recent);
+          else if constexpr (NM_M >= 41 && NM_M <= 43)
             tie |= nm4_fixed<NM_M - 40>(xb, col0 + 64 * bb, pos, p.sink, p.recent, nm_windows);
           else
             tie |= nm_fast<MM>(xb, p.n, col0 + 64 * bb, pos, p.sink, p.recent, nm_windows);
@@ -1131,7 +1160,7 @@ static unsigned long long g_wait_ns = WAIT_TIMEOUT_NS;
 static EncodeTiledFn g_encode = nullptr;
 constexpr int MAX_DEV = 64;
 static int* g_status[MAX_DEV] = {};
-static bool g_attr_set[MAX_DEV][64] = {};
+static bool g_attr_set[MAX_DEV][80] = {};
 
 static EncodeTiledFn encode_fn() {
   if (g_encode) return g_encode;
@@ -1215,18 +1244,20 @@ static int launch_var(const Maps& mp, const Params& p, int grid, cudaStream_t st
 
 template <int D, int BC>
 static int launch(const Maps& mp, const Params& p, int grid, cudaStream_t stream, int dev, int base) {
-  constexpr int PER = 15;  // instances per shape: 5 N:M codes x 3 variants
+  constexpr int PER = 18;  // instances per shape: 6 N:M codes x 3 variants
   if (p.nP > 0) return launch_one<D, BC, 0, 3>(mp, p, grid, stream, dev, 4 * PER + base);
   // N = M keeps every key: the instance without N:M computes exactly that
   const int nm = ((p.mode & SSA_MODE_NM) && p.n < p.m) ? p.m : 0;
-  const int code = nm == 0 ? 0 : nm == 8 ? 1 : 1 + p.n;  // 0 none, 1 eight-wide, 2..4 four-wide N = 1..3
+  // 0 none, 1 eight-wide, 2..4 four-wide N = 1..3, 5 eight-wide N = 4
+  const int code = nm == 0 ? 0 : nm == 8 ? (p.n == 4 ? 5 : 1) : 1 + p.n;
   const int inst = base * PER + 3 * code;
   switch (code) {
     case 0: return launch_var<D, BC, 0>(mp, p, grid, stream, dev, inst);
     case 1: return launch_var<D, BC, 8>(mp, p, grid, stream, dev, inst);
     case 2: return launch_var<D, BC, 41>(mp, p, grid, stream, dev, inst);
     case 3: return launch_var<D, BC, 42>(mp, p, grid, stream, dev, inst);
-    default: return launch_var<D, BC, 43>(mp, p, grid, stream, dev, inst);
+    case 4: return launch_var<D, BC, 43>(mp, p, grid, stream, dev, inst);
+    default: return launch_var<D, BC, 84>(mp, p, grid, stream, dev, inst);
   }
 }
 
