@@ -127,12 +127,12 @@ def _sampled(w, lam, count, keep_bits=False):
 
 @pytest.mark.parametrize("lam", [1e-4, 1e-3, 1e-2])
 def test_llama8k_sampled(lam):
-    rep, _ = _sampled(WORKLOADS["llama8k"], lam, 24)
+    rep, _ = _sampled(WORKLOADS["llama8k"], lam, 64)
     print(rep)
 
 
 def test_llama8k_sink_strong_sampled():
-    rep, _ = _sampled(WORKLOADS["llama8k"].with_(sink_coef=12.0), 1e-3, 24)
+    rep, _ = _sampled(WORKLOADS["llama8k"].with_(sink_coef=12.0), 1e-3, 64)
     assert rep.skipped_gpu > 0
     print(rep)
 
@@ -144,18 +144,18 @@ def test_llama4k_nm_sampled(name):
 
 
 def test_wan_sampled():
-    rep, _ = _sampled(WORKLOADS["wan"], 1e-3, 8)
+    rep, _ = _sampled(WORKLOADS["wan"], 1e-3, 128)
     print(rep)
 
 
 def test_wan_local_sampled():
-    rep, _ = _sampled(WORKLOADS["wan"].with_(local_alpha=2.5), 1e-3, 8)
+    rep, _ = _sampled(WORKLOADS["wan"].with_(local_alpha=2.5), 1e-3, 128)
     assert rep.skipped_gpu > 0
     print(rep)
 
 
 def test_qwen32k_sampled():
     # keep bits of the full problem: B * Hq * Lq * Lk / 32 words (8.6 GB), compared on the sampled items
-    rep, _ = _sampled(WORKLOADS["qwen32k"], 1e-3, 12, keep_bits=True)
+    rep, _ = _sampled(WORKLOADS["qwen32k"], 1e-3, 96, keep_bits=True)
     assert rep.keep_bits_compared > 0
     print(rep)
