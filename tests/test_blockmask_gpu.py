@@ -113,15 +113,16 @@ def test_blockmask_matches_oracle(case):
         assert c.sum() > 0
 
 
-@pytest.mark.parametrize("mode,Br", [(MODE_SKIP, 128), (MODE_SKIP, 64), (MODE_SKIP | MODE_NM, 128)])
-def test_full_mask_reproduces_ssa_fwd(mode, Br):
+@pytest.mark.parametrize("mode,Br,nm", [(MODE_SKIP, 128, None), (MODE_SKIP, 64, None),
+                                        (MODE_SKIP | MODE_NM, 128, (2, 4)), (MODE_SKIP | MODE_NM, 128, (4, 8))])
+def test_full_mask_reproduces_ssa_fwd(mode, Br, nm):
     from softmax_ssa_fwd_b200 import ssa
     q, k, v = _gen(1, 8, 2, 1100, 128, seed=5, sink_coef=12.0)
     qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
     nQ, nK = -(-1100 // Br), -(-1100 // 128)
     full = torch.full((1, 2, nQ, -(-nK // 32)), -1, dtype=torch.int32, device="cuda")
     kw = dict(causal=True, scale=128 ** -0.5, mode=mode, lam=1e-3, Br=Br, Bc=128,
-              n=2 if mode & MODE_NM else 0, m=4 if mode & MODE_NM else 0,
+              n=nm[0] if nm else 0, m=nm[1] if nm else 0,
               sink=4 if mode & MODE_NM else 0, recent=128 if mode & MODE_NM else 0)
     a = ssa.attention_blockmask(qc, kc, vc, full, **kw)
     b = ssa.attention(qc, kc, vc, **kw)

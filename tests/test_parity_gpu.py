@@ -98,10 +98,11 @@ def test_nm_with_n_equal_m_is_dense_bitwise(m):
 
 
 @pytest.mark.parametrize("lam", [1e-3, 3e-2, 1.5])
-def test_skip_combined_with_nm(lam):
+@pytest.mark.parametrize("n,m", [(2, 4), (4, 8)])
+def test_skip_combined_with_nm(lam, n, m):
     q, k, v = _rand(2, 4, 2, 600, 600, 128, seed=9, sink_coef=12.0)
     rep = _full(q, k, v, 128, causal=True, scale=1 / math.sqrt(128), mode=MODE_SKIP | MODE_NM,
-                lam=lam, n=2, m=4, sink=4, recent=128, keep_bits=True)
+                lam=lam, n=n, m=m, sink=4, recent=128, keep_bits=True)
     assert rep.skipped_gpu > 0
 
 
