@@ -94,6 +94,23 @@ struct Params {
   float log2_lambda;  // -inf for lambda == 0
 };
 
+// The prefill TMA load with an L2 cache policy: the K/V stream is read once,
+// and tagging it evict-first keeps the splits' partial results (written
+// meanwhile, read by the combine kernel) in L2.
+__device__ __forceinline__ void tma_load_4d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, int c2, int c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -187,6 +204,7 @@ __global__ void __launch_bounds__(NT, 1)
     if (lane == 0) {
       ssa::tma_prefetch_desc(&tm_k);
       ssa::tma_prefetch_desc(&tm_v);
+      const uint64_t stream_policy = l2_evict_first_policy();
       int g = 0, kdone = 0, vdone = 0;  // tiles walked; K and V tiles issued
       bool ok = true;
       for (int it = blockIdx.x; ok && it < p.n_items; it += gridDim.x) {
@@ -202,7 +220,8 @@ __global__ void __launch_bounds__(NT, 1)
           mbar_arrive_expect_tx(kb, L::TILE_BYTES);
 #pragma unroll
           for (int box = 0; box < D / 64; ++box)
-            ssa::tma_load_4d(k_ring + ks * L::TILE_BYTES + box * BC * 128, &tm_k, kb, box * 64, w.hkv, j0, w.b);
+            tma_load_4d_hint(k_ring + ks * L::TILE_BYTES + box * BC * 128, &tm_k, kb, box * 64, w.hkv, j0, w.b,
+                             stream_policy);
           kdone = g + 1;
           if (!mbar_wait(smem_u32(&vempty[vs]), ((g / VST) & 1) ^ 1, p.wait_ns)) {
             ok = false;
@@ -212,7 +231,8 @@ __global__ void __launch_bounds__(NT, 1)
           mbar_arrive_expect_tx(vb, L::TILE_BYTES);
 #pragma unroll
           for (int box = 0; box < D / 64; ++box)
-            ssa::tma_load_4d(v_ring + vs * L::TILE_BYTES + box * BC * 128, &tm_v, vb, box * 64, w.hkv, j0, w.b);
+            tma_load_4d_hint(v_ring + vs * L::TILE_BYTES + box * BC * 128, &tm_v, vb, box * 64, w.hkv, j0, w.b,
+                             stream_policy);
           vdone = g + 1;
         }
       }
